@@ -1,0 +1,242 @@
+"""Per-step parity of the CUDA kernels against the CPU oracle, through the
+C-ABI single-step entry points (gpt2_op_*). Sizes span several tiles and a
+ragged tail; every tcgen05 tile width is exercised."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from oracle import gpt2_oracle as O
+from tests._cmp import rel_l2, max_abs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def G():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import transformer_decoder_lm_b200 as g   # fails loudly if libgpt2.so is missing
+    return g
+
+
+def dev(a, dtype):
+    td = {"bf16": torch.bfloat16, "fp32": torch.float32, "i32": torch.int32}[dtype]
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda").to(td)
+
+
+def bf16_exact(rng, shape, scale=1.0):
+    return synthetic.round_to_bf16((rng.standard_normal(shape) * scale).astype(np.float32))
+
+
+def status_word():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# ---------------------------------------------------------------- embedding
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_embed(G, dtype):
+    rng = np.random.default_rng(10)
+    V, C, T, Bn = 1000, 768, 37, 3
+    wte = bf16_exact(rng, (V, C), 0.02)
+    wpe = bf16_exact(rng, (64, C), 0.02)
+    ids = rng.integers(0, V, size=(Bn, T)).astype(np.int32)
+    x = torch.empty(Bn * T, C, dtype=torch.float32, device="cuda")
+    st = status_word()
+    code = G.GPT2_BF16 if dtype == "bf16" else G.GPT2_FP32
+    G.gpt2_op_embed(code, dev(ids, "i32"), dev(wte, dtype), dev(wpe, dtype), Bn * T, T, C, V, x, st)
+    ref = O.embed({"wte": wte, "wpe": wpe}, ids).reshape(Bn * T, C)
+    assert max_abs(x.cpu().numpy(), ref) <= 1e-7
+    assert int(st.item()) == 0
+    bad = ids.copy()
+    bad[1, 5] = V + 3
+    G.gpt2_op_embed(code, dev(bad, "i32"), dev(wte, dtype), dev(wpe, dtype), Bn * T, T, C, V, x, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 1                 # recorded, and row 0 was read instead
+    assert np.allclose(x.cpu().numpy()[T + 5], wte[0] + wpe[5], atol=1e-7)
+
+
+# ---------------------------------------------------------------- LayerNorm
+
+
+@pytest.mark.parametrize("C", [64, 768, 1600])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_layernorm(G, dtype, C):
+    rng = np.random.default_rng(C)
+    M = 301
+    x = (rng.standard_normal((M, C)) * 1.7 + 0.4).astype(np.float32)
+    g = (1 + 0.1 * rng.standard_normal(C)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(C)).astype(np.float32)
+    if dtype == "bf16":
+        g, b = synthetic.round_to_bf16(g), synthetic.round_to_bf16(b)
+    out = torch.empty(M, C, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device="cuda")
+    code = G.GPT2_BF16 if dtype == "bf16" else G.GPT2_FP32
+    G.gpt2_op_layernorm(code, dev(x, "fp32"), dev(g, dtype), dev(b, dtype), M, C, out)
+    ref = O.layer_norm(x.astype(np.float64), g, b)
+    got = out.float().cpu().numpy()
+    if dtype == "fp32":
+        assert max_abs(got, ref) <= 2e-5
+    else:
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5)
+
+
+# ------------------------------------------------------------------- Linear
+
+LINEAR_SHAPES = [
+    (300, 2304, 768),     # c_attn-like, ragged M
+    (128, 200, 64),       # one m-tile, N tail inside a 64-column group
+    (515, 776, 256),      # N tail past 768
+    (64, 1600, 1600),     # partial m-tile only
+]
+
+
+@pytest.mark.parametrize("bn", ["64", "128", "256", ""])
+@pytest.mark.parametrize("epi", [0, 1, 2])
+@pytest.mark.parametrize("shape", LINEAR_SHAPES)
+def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
+    if bn:
+        monkeypatch.setenv("G2_GEMM_BN", bn)
+    else:
+        monkeypatch.delenv("G2_GEMM_BN", raising=False)
+    M, N, K = shape
+    rng = np.random.default_rng(M * 7 + N + K + epi)
+    A = bf16_exact(rng, (M, K))
+    W = bf16_exact(rng, (N, K), 1.0 / math.sqrt(K))
+    bias = bf16_exact(rng, (N,), 0.1)
+    st = status_word()
+    ref = O.linear(A.astype(np.float64), W.astype(np.float64), bias.astype(np.float64))
+    if epi == 2:
+        x0 = rng.standard_normal((M, N)).astype(np.float32)
+        out = dev(x0, "fp32")
+        ref = ref + x0
+    else:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        if epi == 1:
+            ref = O.gelu(ref)
+    G.gpt2_op_linear(G.GPT2_BF16, epi, dev(A, "bf16"), dev(W, "bf16"), dev(bias, "bf16"), M, N, K, out, st)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    assert int(st.item()) == 0
+    if epi == 2:
+        assert max_abs(got, ref) <= 1e-4 * max(1.0, math.sqrt(K) / 16)
+    else:
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-4)
+
+
+@pytest.mark.parametrize("epi", [0, 1, 2])
+def test_linear_fp32_simt(G, epi):
+    M, N, K = 130, 200, 72
+    rng = np.random.default_rng(40 + epi)
+    A = rng.standard_normal((M, K)).astype(np.float32)
+    W = rng.standard_normal((N, K)).astype(np.float32) / math.sqrt(K)
+    bias = rng.standard_normal(N).astype(np.float32) * 0.1
+    ref = O.linear(A.astype(np.float64), W.astype(np.float64), bias.astype(np.float64))
+    if epi == 2:
+        x0 = rng.standard_normal((M, N)).astype(np.float32)
+        out = dev(x0, "fp32")
+        ref = ref + x0
+    else:
+        out = torch.empty(M, N, dtype=torch.float32, device="cuda")
+        if epi == 1:
+            ref = O.gelu(ref)
+    G.gpt2_op_linear(G.GPT2_FP32, epi, dev(A, "fp32"), dev(W, "fp32"), dev(bias, "fp32"), M, N, K, out)
+    assert max_abs(out.cpu().numpy(), ref) <= 2e-5
+
+
+# ---------------------------------------------------------------- attention
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("B,T,H,C", [(2, 200, 4, 256), (1, 64, 2, 64), (3, 1, 12, 768), (1, 333, 12, 768)])
+def test_attention(G, dtype, B, T, H, C):
+    rng = np.random.default_rng(B * 1000 + T + H)
+    qkv = bf16_exact(rng, (B * T, 3 * C))
+    y = torch.empty(B * T, C, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device="cuda")
+    code = G.GPT2_BF16 if dtype == "bf16" else G.GPT2_FP32
+    G.gpt2_op_attention(code, dev(qkv, dtype), B, T, H, C, y)
+    ref = O.causal_self_attention(qkv.astype(np.float64).reshape(B, T, 3 * C), H).reshape(B * T, C)
+    got = y.float().cpu().numpy()
+    if dtype == "fp32":
+        assert max_abs(got, ref) <= 1e-5
+    else:
+        assert rel_l2(got, ref) <= 5e-3
+        assert max_abs(got, ref) <= 2e-2
+
+
+# ------------------------------------------------------- lm_head + cross-entropy
+
+
+@pytest.mark.parametrize("bn", ["64", "128", "256", ""])
+@pytest.mark.parametrize("M,C,V", [(300, 768, 1000), (128, 128, 50257)])
+def test_lmhead_ce_bf16(G, M, C, V, bn, monkeypatch):
+    if bn:
+        monkeypatch.setenv("G2_GEMM_BN", bn)
+    else:
+        monkeypatch.delenv("G2_GEMM_BN", raising=False)
+    rng = np.random.default_rng(M + C + V)
+    hf = bf16_exact(rng, (M, C))
+    wte = bf16_exact(rng, (V, C), 0.05)
+    targets = rng.integers(0, V, size=M).astype(np.int32)
+    targets[::7] = -1                         # ignored positions
+    targets[3] = V - 1                        # last real column (inside the padded tile)
+    ws = torch.empty(G.gpt2_op_lmhead_ce_workspace_bytes(G.GPT2_BF16, M, V), dtype=torch.uint8, device="cuda")
+    logits = torch.empty(M, V, dtype=torch.float32, device="cuda")
+    tok = torch.empty(M, dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    st = status_word()
+    G.gpt2_op_lmhead_ce(G.GPT2_BF16, dev(hf, "bf16"), dev(wte, "bf16"), dev(targets, "i32"), M, C, V, logits, tok,
+                        loss, ws, st)
+    torch.cuda.synchronize()
+    z = hf.astype(np.float64) @ wte.astype(np.float64).T
+    lse = O.logsumexp_last(z)
+    valid = targets >= 0
+    ref_tok = np.where(valid, lse - z[np.arange(M), np.maximum(targets, 0)], 0.0)
+    assert int(st.item()) == 0
+    assert max_abs(logits.cpu().numpy(), z) <= 1e-4 * math.sqrt(C) / 8
+    assert max_abs(tok.cpu().numpy(), ref_tok) <= 1e-4
+    assert abs(float(loss.item()) - ref_tok[valid].mean()) <= 1e-5
+    # loss-only call (no logits) gives the same losses
+    tok2 = torch.empty_like(tok)
+    G.gpt2_op_lmhead_ce(G.GPT2_BF16, dev(hf, "bf16"), dev(wte, "bf16"), dev(targets, "i32"), M, C, V, None, tok2,
+                        loss, ws, st)
+    assert torch.equal(tok, tok2)
+
+
+def test_lmhead_ce_fp32(G):
+    M, C, V = 70, 64, 512
+    rng = np.random.default_rng(3)
+    hf = rng.standard_normal((M, C)).astype(np.float32)
+    wte = (rng.standard_normal((V, C)) * 0.1).astype(np.float32)
+    targets = rng.integers(-1, V, size=M).astype(np.int32)
+    ws = torch.empty(G.gpt2_op_lmhead_ce_workspace_bytes(G.GPT2_FP32, M, V), dtype=torch.uint8, device="cuda")
+    logits = torch.empty(M, V, dtype=torch.float32, device="cuda")
+    tok = torch.empty(M, dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    G.gpt2_op_lmhead_ce(G.GPT2_FP32, dev(hf, "fp32"), dev(wte, "fp32"), dev(targets, "i32"), M, C, V, logits, tok,
+                        loss, ws)
+    z = hf.astype(np.float64) @ wte.astype(np.float64).T
+    lse = O.logsumexp_last(z)
+    valid = targets >= 0
+    ref_tok = np.where(valid, lse - z[np.arange(M), np.maximum(targets, 0)], 0.0)
+    assert max_abs(logits.cpu().numpy(), z) <= 1e-5
+    assert max_abs(tok.cpu().numpy(), ref_tok) <= 1e-5
+    assert abs(float(loss.item()) - ref_tok[valid].mean()) <= 1e-6
+
+
+def test_lmhead_ce_no_targets_sets_status(G):
+    M, C, V = 16, 64, 100
+    hf = torch.zeros(M, C, dtype=torch.float32, device="cuda")
+    wte = torch.zeros(V, C, dtype=torch.float32, device="cuda")
+    tg = torch.full((M,), -1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(G.gpt2_op_lmhead_ce_workspace_bytes(G.GPT2_FP32, M, V), dtype=torch.uint8, device="cuda")
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    st = status_word()
+    G.gpt2_op_lmhead_ce(G.GPT2_FP32, hf, wte, tg, M, C, V, None, None, loss, ws, st)
+    torch.cuda.synchronize()
+    assert math.isnan(float(loss.item()))
+    assert int(st.item()) & 4

@@ -1,0 +1,207 @@
+"""ctypes binding of libgpt2.so (include/gpt2.h), argument marshalling only.
+
+Every function here has the name of the C entry point it calls and takes
+torch tensors (device memory owned by the caller) or plain integers; it
+converts them to pointers and sizes, calls the library, and raises
+``GPT2Error`` on a non-zero return code. All computation happens in the CUDA
+kernels of libgpt2.so: there is no fallback of any kind, and importing this
+module fails loudly if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgpt2.so")
+
+GPT2_BF16, GPT2_FP32 = 0, 1
+GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID = 0, 1, 2
+ERRORS = {
+    0: "GPT2_OK", 1: "GPT2_ERR_INVALID_ARG", 2: "GPT2_ERR_UNSUPPORTED", 3: "GPT2_ERR_CUDA",
+    4: "GPT2_ERR_WORKSPACE", 5: "GPT2_ERR_BAD_TOKEN", 6: "GPT2_ERR_DEVICE_TIMEOUT", 7: "GPT2_ERR_NO_TARGETS",
+}
+ERR_CODE = {v: k for k, v in ERRORS.items()}
+
+LAYER_KEYS = (
+    "ln1_g", "ln1_b", "attn_w", "attn_b", "attn_proj_w", "attn_proj_b",
+    "ln2_g", "ln2_b", "fc_w", "fc_b", "mlp_proj_w", "mlp_proj_b",
+)
+
+
+class GPT2Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {ERRORS.get(code, code)} ({code})")
+
+
+class gpt2_config_t(ctypes.Structure):
+    _fields_ = [("n_layer", ctypes.c_int), ("n_head", ctypes.c_int), ("n_embd", ctypes.c_int),
+                ("vocab", ctypes.c_int), ("n_ctx", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("flags", ctypes.c_uint)]
+
+
+_PP = ctypes.POINTER(ctypes.c_void_p)
+
+
+class gpt2_weights_t(ctypes.Structure):
+    _fields_ = [("wte", ctypes.c_void_p), ("wpe", ctypes.c_void_p)] + \
+               [(k, _PP) for k in LAYER_KEYS] + \
+               [("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libgpt2.so is not built ({LIB_PATH}); run python transformer_decoder_lm_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "gpt2_workspace_bytes": (sz, [ctypes.POINTER(gpt2_config_t), i, i]),
+        "gpt2_create": (i, [ctypes.POINTER(gpt2_config_t), ctypes.POINTER(gpt2_weights_t), vp, sz, i, i,
+                            ctypes.POINTER(vp)]),
+        "gpt2_forward": (i, [vp, vp, i, i, vp, vp]),
+        "gpt2_loss": (i, [vp, vp, vp, i, i, vp, vp]),
+        "gpt2_forward_loss": (i, [vp, vp, vp, i, i, vp, vp, vp, vp]),
+        "gpt2_status": (i, [vp, vp]),
+        "gpt2_error_string": (ctypes.c_char_p, [i]),
+        "gpt2_destroy": (None, [vp]),
+        "gpt2_launch_count": (ctypes.c_uint64, [vp]),
+        "gpt2_set_timing_events": (i, [vp, i, vp, vp]),
+        "gpt2_op_embed": (i, [i, vp, vp, vp, i, i, i, i, vp, vp, vp]),
+        "gpt2_op_layernorm": (i, [i, vp, vp, vp, i, i, vp, vp]),
+        "gpt2_op_linear": (i, [i, i, vp, vp, vp, i, i, i, vp, vp, vp]),
+        "gpt2_op_attention": (i, [i, vp, i, i, i, i, vp, vp, vp]),
+        "gpt2_op_lmhead_ce_workspace_bytes": (sz, [i, i, i]),
+        "gpt2_op_lmhead_ce": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib, sig
+
+
+lib, SIGNATURES = _load()
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise GPT2Error(rc, where)
+
+
+def make_config(n_layer: int, n_head: int, n_embd: int, vocab: int, n_ctx: int, dtype: int) -> gpt2_config_t:
+    return gpt2_config_t(n_layer, n_head, n_embd, vocab, n_ctx, dtype, 0)
+
+
+def gpt2_workspace_bytes(cfg: gpt2_config_t, max_B: int, max_T: int) -> int:
+    return int(lib.gpt2_workspace_bytes(ctypes.byref(cfg), max_B, max_T))
+
+
+class _Weights:
+    """Keeps the ctypes pointer arrays alive as long as the handle."""
+
+    def __init__(self, w: Dict[str, object]):
+        n = len(w["layers"])
+        self.arrays = {k: (ctypes.c_void_p * n)(*[_ptr(lw[k]) for lw in w["layers"]]) for k in LAYER_KEYS}
+        self.struct = gpt2_weights_t(
+            _ptr(w["wte"]), _ptr(w["wpe"]),
+            *[ctypes.cast(self.arrays[k], _PP) for k in LAYER_KEYS],
+            _ptr(w["lnf_g"]), _ptr(w["lnf_b"]))
+
+
+def gpt2_create(cfg: gpt2_config_t, weights: Dict[str, object], workspace, max_B: int, max_T: int):
+    """weights: {'wte','wpe','lnf_g','lnf_b': tensor, 'layers': [ {LAYER_KEYS: tensor} ]}
+    (device tensors of cfg.dtype). Returns (handle, keepalive)."""
+    keep = _Weights(weights)
+    h = ctypes.c_void_p()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.gpt2_create(ctypes.byref(cfg), ctypes.byref(keep.struct), _ptr(workspace), nbytes, max_B, max_T,
+                           ctypes.byref(h)), "gpt2_create")
+    return h, keep
+
+
+def gpt2_forward(h, ids, B: int, T: int, logits=None, stream=None) -> None:
+    _check(lib.gpt2_forward(h, _ptr(ids), B, T, _ptr(logits), _stream(stream)), "gpt2_forward")
+
+
+def gpt2_loss(h, ids, targets, B: int, T: int, loss_out, stream=None) -> None:
+    _check(lib.gpt2_loss(h, _ptr(ids), _ptr(targets), B, T, _ptr(loss_out), _stream(stream)), "gpt2_loss")
+
+
+def gpt2_forward_loss(h, ids, targets, B: int, T: int, logits, loss_out, token_loss=None, stream=None) -> None:
+    _check(lib.gpt2_forward_loss(h, _ptr(ids), _ptr(targets), B, T, _ptr(logits), _ptr(loss_out), _ptr(token_loss),
+                                 _stream(stream)), "gpt2_forward_loss")
+
+
+def gpt2_status(h, stream=None) -> int:
+    return int(lib.gpt2_status(h, _stream(stream)))
+
+
+def gpt2_error_string(code: int) -> str:
+    return lib.gpt2_error_string(code).decode()
+
+
+def gpt2_destroy(h) -> None:
+    lib.gpt2_destroy(h)
+
+
+def gpt2_launch_count(h) -> int:
+    return int(lib.gpt2_launch_count(h))
+
+
+GPT2_TIMED_LMHEAD = 0
+
+
+def gpt2_set_timing_events(h, which: int, ev_begin=None, ev_end=None) -> None:
+    """ev_begin / ev_end: torch.cuda.Event (created with enable_timing=True) or None."""
+    b = ev_begin.cuda_event if ev_begin is not None else None
+    e = ev_end.cuda_event if ev_end is not None else None
+    _check(lib.gpt2_set_timing_events(h, which, b, e), "gpt2_set_timing_events")
+
+
+def gpt2_op_embed(dtype, ids, wte, wpe, M, T, C, V, x, status=None, stream=None):
+    _check(lib.gpt2_op_embed(dtype, _ptr(ids), _ptr(wte), _ptr(wpe), M, T, C, V, _ptr(x), _ptr(status),
+                             _stream(stream)), "gpt2_op_embed")
+
+
+def gpt2_op_layernorm(dtype, x, g, b, M, C, out, stream=None):
+    _check(lib.gpt2_op_layernorm(dtype, _ptr(x), _ptr(g), _ptr(b), M, C, _ptr(out), _stream(stream)),
+           "gpt2_op_layernorm")
+
+
+def gpt2_op_linear(dtype, epilogue, A, W, bias, M, N, K, out, status=None, stream=None):
+    _check(lib.gpt2_op_linear(dtype, epilogue, _ptr(A), _ptr(W), _ptr(bias), M, N, K, _ptr(out), _ptr(status),
+                              _stream(stream)), "gpt2_op_linear")
+
+
+def gpt2_op_attention(dtype, qkv, B, T, H, C, y, status=None, stream=None):
+    _check(lib.gpt2_op_attention(dtype, _ptr(qkv), B, T, H, C, _ptr(y), _ptr(status), _stream(stream)),
+           "gpt2_op_attention")
+
+
+def gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V) -> int:
+    return int(lib.gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V))
+
+
+def gpt2_op_lmhead_ce(dtype, hf, wte, targets, M, C, V, logits, token_loss, loss_out, workspace, status=None,
+                      stream=None):
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.gpt2_op_lmhead_ce(dtype, _ptr(hf), _ptr(wte), _ptr(targets), M, C, V, _ptr(logits), _ptr(token_loss),
+                                 _ptr(loss_out), _ptr(workspace), nbytes, _ptr(status), _stream(stream)),
+           "gpt2_op_lmhead_ce")

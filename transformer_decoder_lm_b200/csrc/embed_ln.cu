@@ -1,0 +1,160 @@
+// embed_ln.cu - embedding sum and LayerNorm kernels (HBM-bound, SIMT).
+//
+// embed:      x[m, :] = wte[ids[m], :] + wpe[m % T, :]        fp32 residual stream
+//             ("Hand-writing GPT-2 from scratch: the Transformer decoder core
+//              modules in PyTorch", section 4.1 forward step 1).
+// layernorm:  out[m, :] = (x - mean) * rsqrt(var_biased + 1e-5) * g + b
+//             ("Reproducing GPT-2 124M", section 2.1, hand-written LayerNorm with
+//              unbiased=False; eps 1e-5 per the first page, sections 3.2/4.2).
+//
+// Both kernels give each row to one warp and move 16-byte (fp32) or 8-byte
+// (bf16) vectors; the row stays in registers between the two passes of the
+// LayerNorm statistics (mean, then the centred second moment), so x is read
+// from HBM exactly once.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace g2 {
+
+template <typename T>
+struct Vec4;
+template <>
+struct Vec4<float> {
+  static __device__ __forceinline__ float4 load(const float* p) { return *reinterpret_cast<const float4*>(p); }
+  static __device__ __forceinline__ void store(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+};
+template <>
+struct Vec4<bf16> {
+  static __device__ __forceinline__ float4 load(const bf16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+  }
+  static __device__ __forceinline__ void store(bf16* p, float4 v) {
+    uint2 u;
+    u.x = pack_bf16x2(v.x, v.y);
+    u.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids, const T* __restrict__ wte,
+                                                    const T* __restrict__ wpe, float* __restrict__ x, int M,
+                                                    int Tlen, int C, int V, int* status) {
+  const int warps = blockDim.x >> 5;
+  const int row = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  int id = ids[row];
+  if (id < 0 || id >= V) {
+    if (lane == 0) record_error(status, DEV_BAD_TOKEN);
+    id = 0;
+  }
+  const int t = row % Tlen;
+  const T* te = wte + (size_t)id * C;
+  const T* pe = wpe + (size_t)t * C;
+  float* xr = x + (size_t)row * C;
+  for (int c = lane * 4; c < C; c += 128) {
+    const float4 a = Vec4<T>::load(te + c);
+    const float4 b = Vec4<T>::load(pe + c);
+    Vec4<float>::store(xr + c, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// C <= 32 lanes * 4 * MAXV = 2048.
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, const T* __restrict__ g,
+                                                        const T* __restrict__ b, T* __restrict__ out, int M,
+                                                        int C) {
+  const int warps = blockDim.x >> 5;
+  const int row = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float* xr = x + (size_t)row * C;
+  float4 v[MAXV];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) {
+      v[i] = Vec4<float>::load(xr + c);
+      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    }
+  }
+  const float mean = warp_sum(s) / (float)C;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) {
+      const float a = v[i].x - mean, bb = v[i].y - mean, cc = v[i].z - mean, d = v[i].w - mean;
+      q += (a * a + bb * bb) + (cc * cc + d * d);
+    }
+  }
+  const float var = warp_sum(q) / (float)C;
+  const float rstd = rsqrtf(var + 1e-5f);
+  T* orow = out + (size_t)row * C;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) {
+      const float4 gg = Vec4<T>::load(g + c);
+      const float4 bt = Vec4<T>::load(b + c);
+      float4 o;
+      o.x = (v[i].x - mean) * rstd * gg.x + bt.x;
+      o.y = (v[i].y - mean) * rstd * gg.y + bt.y;
+      o.z = (v[i].z - mean) * rstd * gg.z + bt.z;
+      o.w = (v[i].w - mean) * rstd * gg.w + bt.w;
+      Vec4<T>::store(orow + c, o);
+    }
+  }
+}
+
+cudaError_t embed_launch(bool bf16_, const int* ids, const void* wte, const void* wpe, float* x, int M, int T,
+                         int C, int V, int* status, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  const int threads = 256, rows_per_block = threads / 32;
+  const int grid = (M + rows_per_block - 1) / rows_per_block;
+  if (bf16_)
+    embed_kernel<bf16><<<grid, threads, 0, s>>>(ids, static_cast<const bf16*>(wte), static_cast<const bf16*>(wpe),
+                                                 x, M, T, C, V, status);
+  else
+    embed_kernel<float><<<grid, threads, 0, s>>>(ids, static_cast<const float*>(wte),
+                                                  static_cast<const float*>(wpe), x, M, T, C, V, status);
+  return cudaGetLastError();
+}
+
+cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const void* b, void* out, int M, int C,
+                             cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (C > 2048 || (C & 3)) return cudaErrorInvalidValue;
+  const int threads = 256, rows_per_block = threads / 32;
+  const int grid = (M + rows_per_block - 1) / rows_per_block;
+  if (bf16_) {
+    if (C <= 1024)
+      layernorm_kernel<bf16, 8><<<grid, threads, 0, s>>>(x, static_cast<const bf16*>(g), static_cast<const bf16*>(b),
+                                                         static_cast<bf16*>(out), M, C);
+    else
+      layernorm_kernel<bf16, 16><<<grid, threads, 0, s>>>(x, static_cast<const bf16*>(g),
+                                                          static_cast<const bf16*>(b), static_cast<bf16*>(out), M, C);
+  } else {
+    if (C <= 1024)
+      layernorm_kernel<float, 8><<<grid, threads, 0, s>>>(x, static_cast<const float*>(g),
+                                                          static_cast<const float*>(b), static_cast<float*>(out), M, C);
+    else
+      layernorm_kernel<float, 16><<<grid, threads, 0, s>>>(x, static_cast<const float*>(g),
+                                                           static_cast<const float*>(b), static_cast<float*>(out), M,
+                                                           C);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace g2

@@ -1,0 +1,446 @@
+// gemm_tc.cu - tcgen05 / TMEM / TMA GEMM with fused epilogues (sm_100a).
+//
+// Computes C = A . B^T for the four Linear layers of a GPT-2 block and the
+// tied lm_head ("Hand-writing GPT-2 from scratch: the Transformer decoder
+// core modules in PyTorch", sections 2.2 and 3.4; "Reproducing GPT-2 124M",
+// section 2.1: c_attn, c_proj, c_fc, c_proj and lm_head = wte^T), in bf16
+// with fp32 accumulation, A [M, K] and B [N, K] both K-major (the
+// nn.Linear [out, in] layout is already the K-major B operand).
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: 128x64 A box and BNx64 B box per stage, 128-byte
+//               swizzle, STAGES-deep ring of shared-memory stages.
+//   warp 1      allocates 2*BN TMEM columns and issues tcgen05.mma
+//               (M=128, N=BN, K=16, four per 64-wide k-block) into one of two
+//               TMEM accumulators; tcgen05.commit frees smem stages and hands
+//               finished accumulators to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, 32 columns at a
+//               time, fused bias / GELU(erf) / residual add / log-sum-exp.
+// The double-buffered accumulator lets the epilogue of tile i overlap the
+// main loop of tile i+1. Tiles are walked M-fastest so that consecutive CTAs
+// share the B tile in L2 (the 77 MB wte of the lm_head is streamed ~once).
+//
+// The lm_head epilogue never needs the logits in HBM: per row and column
+// tile it emits (max, sum exp(z - max)) and, in the tile holding the target
+// column, the target logit; a small kernel finishes the log-sum-exp.
+// Columns at or past N (the vocabulary padded up to the tile width by TMA
+// zero fill) are excluded from the sums and from the logits.
+//
+// Every wait is bounded (common.cuh): on a timeout the kernel records
+// GPT2_ERR_DEVICE_TIMEOUT, lets its in-flight copies and MMAs land, frees its
+// TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <stdlib.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace g2 {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BK = 64;
+constexpr int TC_THREADS = 192;
+constexpr int STAGING_FLOATS = 4 * 32 * 33;   // per-warp 32x33 transposition buffers (lm_head logits)
+
+template <int BN, int STAGES>
+struct TcLayout {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGING_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFFSET = STAGING_OFFSET + STAGING_FLOATS * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
+  static constexpr int SMEM_BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + tmem holder, abort flag, align slack
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
+};
+
+__device__ __forceinline__ float bf2f(const bf16 v) { return __bfloat162float(v); }
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs args) {
+  using L = TcLayout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* staging = reinterpret_cast<float*>(smem + L::STAGING_OFFSET);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int M = args.M, N = args.N;
+  const int m_tiles = (M + TC_BM - 1) / TC_BM;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int nk = args.K / TC_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_parity = 0;   // per stage: a load was issued / its barrier phase parity
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % m_tiles) * TC_BM;
+        const int n0 = (tile / m_tiles) * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * L::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, &full[stage], kb * TC_BK, m0);
+          tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * TC_BK, n0);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        record_error(args.status, DEV_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // Let every issued copy land before the CTA can exit (bounded).
+      volatile int no_abort = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) mbar_wait(&full[s], (issued_parity >> s) & 1u, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
+          const uint64_t adesc = sdesc_kmajor_sw128(sa);
+          const uint64_t bdesc = sdesc_kmajor_sw128(sa + L::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k)
+            mma_bf16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0);
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        record_error(args.status, DEV_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // Every MMA issued above has completed once `drain` flips.
+      mma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;   // TMEM lane quadrant this warp may access
+    float* stg = staging + q * (32 * 33);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+        if (lane == 0) {
+          record_error(args.status, DEV_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
+      const int row = m0 + q * 32 + lane;
+      const bool row_ok = row < M;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+
+      float run_max = -INFINITY, run_sum = 0.f, tgt_val = 0.f;
+      int tgt = -1;
+      if (EPI == EPI_LMHEAD) tgt = (row_ok && args.targets != nullptr) ? args.targets[row] : -1;
+
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = n0 + c * 32;
+        if (col0 >= N) break;   // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, r);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+
+        if (EPI == EPI_BIAS || EPI == EPI_GELU) {
+          const bf16* bias = static_cast<const bf16*>(args.bias);
+          bf16* o = static_cast<bf16*>(args.out) + (size_t)row * args.ldo + col0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = col0 + g * 8;
+            if (row_ok && col < N) {
+              const uint4 bw = *reinterpret_cast<const uint4*>(bias + col);
+              const bf16* bb = reinterpret_cast<const bf16*>(&bw);
+              float t[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                t[j] = v[g * 8 + j] + bf2f(bb[j]);
+                if (EPI == EPI_GELU) t[j] = gelu_erf(t[j]);
+              }
+              uint4 pk;
+              pk.x = pack_bf16x2(t[0], t[1]);
+              pk.y = pack_bf16x2(t[2], t[3]);
+              pk.z = pack_bf16x2(t[4], t[5]);
+              pk.w = pack_bf16x2(t[6], t[7]);
+              *reinterpret_cast<uint4*>(o + g * 8) = pk;
+            }
+          }
+        } else if (EPI == EPI_RESID) {
+          const bf16* bias = static_cast<const bf16*>(args.bias);
+          float* o = static_cast<float*>(args.out) + (size_t)row * args.ldo + col0;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const int col = col0 + g * 4;
+            if (row_ok && col < N) {
+              const uint2 bw = *reinterpret_cast<const uint2*>(bias + col);
+              const bf16* bb = reinterpret_cast<const bf16*>(&bw);
+              float4 x = *reinterpret_cast<float4*>(o + g * 4);
+              x.x += v[g * 4 + 0] + bf2f(bb[0]);
+              x.y += v[g * 4 + 1] + bf2f(bb[1]);
+              x.z += v[g * 4 + 2] + bf2f(bb[2]);
+              x.w += v[g * 4 + 3] + bf2f(bb[3]);
+              *reinterpret_cast<float4*>(o + g * 4) = x;
+            }
+          }
+        } else {  // EPI_LMHEAD
+          const int nvalid = min(32, N - col0);
+          float cmax = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nvalid) cmax = fmaxf(cmax, v[j]);
+          const float new_max = fmaxf(run_max, cmax);
+          constexpr float LOG2E = 1.4426950408889634f;
+          const float nm2 = new_max * LOG2E;
+          float s = run_sum * exp2f(run_max * LOG2E - nm2);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j < nvalid) s += exp2f(fmaf(v[j], LOG2E, -nm2));
+            if (col0 + j == tgt) tgt_val = v[j];
+          }
+          run_sum = s;
+          run_max = new_max;
+          if (args.out != nullptr) {
+            // Transpose through shared memory so that each row segment is
+            // written by 32 consecutive lanes (the logits row pitch V is odd,
+            // so rows are only 4-byte aligned).
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = v[j];
+            __syncwarp();
+            float* lg = static_cast<float*>(args.out);
+            const int gcol = col0 + lane;
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+              const int grow = m0 + q * 32 + rr;
+              if (grow < M && gcol < N) lg[(size_t)grow * args.ldo + gcol] = stg[rr * 33 + lane];
+            }
+            __syncwarp();
+          }
+        }
+      }
+      // Accumulator fully read: hand it back to the MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+
+      if (EPI == EPI_LMHEAD && row_ok) {
+        args.part[(size_t)n_blk * M + row] = make_float2(run_max, run_sum);
+        if (tgt >= n0 && tgt < n0 + BN && tgt < N) args.tgt_logit[row] = tgt_val;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool load_encode() {
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+template <int BN>
+constexpr int stages_for() {
+  return BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+}
+
+template <int BN, int EPI>
+cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& a, int num_sms,
+                       cudaStream_t s) {
+  constexpr int ST = stages_for<BN>();
+  using L = TcLayout<BN, ST>;
+  const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
+  const int grid = std::min(tiles, num_sms);
+  if (grid <= 0) return cudaSuccess;
+  gemm_tc_kernel<BN, ST, EPI><<<grid, TC_THREADS, L::SMEM_BYTES, s>>>(tA, tB, a);
+  return cudaGetLastError();
+}
+
+template <int BN, int EPI>
+cudaError_t set_attr_one() {
+  constexpr int ST = stages_for<BN>();
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, ST, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcLayout<BN, ST>::SMEM_BYTES);
+}
+
+template <int BN>
+cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& a, int num_sms,
+                      cudaStream_t s) {
+  switch (epi) {
+    case EPI_BIAS: return launch_one<BN, EPI_BIAS>(tA, tB, a, num_sms, s);
+    case EPI_GELU: return launch_one<BN, EPI_GELU>(tA, tB, a, num_sms, s);
+    case EPI_RESID: return launch_one<BN, EPI_RESID>(tA, tB, a, num_sms, s);
+    case EPI_LMHEAD: return launch_one<BN, EPI_LMHEAD>(tA, tB, a, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                    uint32_t box_rows) {
+  if (!load_encode()) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15) || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int gemm_tc_n_tiles(int N, int bn) { return (N + bn - 1) / bn; }
+
+int gemm_tc_pick_bn(int M, int N, int num_sms) {
+  // G2_GEMM_BN=64|128|256 pins the tile width (tests use it to cover every
+  // instantiation); otherwise the width is chosen by the cost model below.
+  if (const char* e = getenv("G2_GEMM_BN")) {
+    const int v = atoi(e);
+    if (v == 64 || v == 128 || v == 256) return v;
+  }
+  // Estimated cost = waves x per-tile cost. Narrow tiles re-read A from shared
+  // memory more often per FLOP, so their per-column cost is higher.
+  const int cand[3] = {256, 128, 64};
+  const double unit[3] = {256.0, 136.0, 96.0};
+  const int mt = (M + TC_BM - 1) / TC_BM;
+  int best = 256;
+  double best_cost = 1e30;
+  for (int i = 0; i < 3; ++i) {
+    const long tiles = (long)mt * ((N + cand[i] - 1) / cand[i]);
+    const long waves = (tiles + num_sms - 1) / num_sms;
+    const double cost = waves * unit[i];
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = cand[i];
+    }
+  }
+  return best;
+}
+
+cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& a,
+                           int num_sms, cudaStream_t s) {
+  switch (bn) {
+    case 256: return launch_bn<256>(epi, tA, tB, a, num_sms, s);
+    case 128: return launch_bn<128>(epi, tA, tB, a, num_sms, s);
+    case 64: return launch_bn<64>(epi, tA, tB, a, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t gemm_tc_set_attributes() {
+  cudaError_t e = cudaSuccess;
+#define G2_ATTR(BN)                                              \
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_BIAS>();        \
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU>();        \
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID>();       \
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD>();
+  G2_ATTR(256)
+  G2_ATTR(128)
+  G2_ATTR(64)
+#undef G2_ATTR
+  return e;
+}
+
+}  // namespace g2

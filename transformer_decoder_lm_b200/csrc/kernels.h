@@ -1,0 +1,61 @@
+// kernels.h - host-side launchers of the forward-pass kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace g2 {
+
+// Epilogues of the Linear layers (values match the public GPT2_EPI_*),
+// plus the fused lm_head / cross-entropy epilogue.
+enum EpiKind : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_LMHEAD = 3 };
+
+struct GemmArgs {
+  int M, N, K;
+  const void* bias;        // [N] of the operand dtype (NULL for the lm_head)
+  void* out;               // EPI_BIAS/GELU: [M, ldo] operand dtype; EPI_RESID: fp32 [M, ldo] (+=);
+                           // EPI_LMHEAD: fp32 logits [M, ldo] or NULL
+  long long ldo;
+  const int* targets;      // EPI_LMHEAD: [M]
+  float2* part;            // EPI_LMHEAD: per (column tile, row) (max, sum exp(z - max)), [n_tiles, M]
+  float* tgt_logit;        // EPI_LMHEAD: [M] logit of the target column
+  int* status;
+};
+
+// ---- tensor maps (host) -------------------------------------------------
+// Encode a 2-D bf16 row-major tensor [rows, cols] (row pitch `ld` elements)
+// read in boxes of box_rows x 64 columns with 128-byte swizzling.
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                    uint32_t box_rows);
+
+// ---- tcgen05 GEMM (bf16) -------------------------------------------------
+// C = A[M,K] . B[N,K]^T with the epilogue `epi`. K % 64 == 0, N % 8 == 0.
+// tmA: box 128 x 64 over A; tmB: box BN x 64 over B, BN from gemm_tc_pick_bn.
+int gemm_tc_pick_bn(int M, int N, int num_sms);
+cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                           const GemmArgs& a, int num_sms, cudaStream_t s);
+cudaError_t gemm_tc_set_attributes();
+int gemm_tc_n_tiles(int N, int bn);
+
+// ---- SIMT fp32 GEMM (fp32 mode) ------------------------------------------
+constexpr int SIMT_BN = 64;
+cudaError_t gemm_simt_launch(int epi, const float* A, const float* W, const GemmArgs& a, cudaStream_t s);
+
+// ---- embedding / LayerNorm -------------------------------------------------
+cudaError_t embed_launch(bool bf16, const int* ids, const void* wte, const void* wpe, float* x, int M, int T,
+                         int C, int V, int* status, cudaStream_t s);
+cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const void* b, void* out, int M, int C,
+                             cudaStream_t s);
+
+// ---- attention ---------------------------------------------------------------
+cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C, int* status,
+                             cudaStream_t s);
+
+// ---- cross-entropy finalisation -------------------------------------------
+// token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
+// target is negative); loss_out (if not NULL) = mean over scored rows.
+cudaError_t ce_finish_launch(const float2* part, int n_tiles, const float* tgt_logit, const int* targets, int M,
+                             int V, float* token_loss, float* loss_out, int* status, cudaStream_t s);
+
+}  // namespace g2
