@@ -312,15 +312,75 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_kernel(args):
+    """Run one step of the forward pass on its own, at the 124M workload's
+    shapes, through the single-step C entry points (for per-kernel timing and
+    profiler captures). Prints the mean CUDA-event time per launch."""
+    import torch
+    import transformer_decoder_lm_b200 as G
+
+    torch.cuda.set_device(0)
+    rng = np.random.default_rng(0)
+    M, C, V, H = WL.batch * WL.seq, WL.n_embd, WL.vocab, WL.n_head
+    bf = torch.bfloat16
+
+    def rnd(*shape, scale=1.0, dtype=bf):
+        return (torch.from_numpy(rng.standard_normal(shape).astype(np.float32)) * scale).to("cuda", dtype)
+
+    k = args.kernel
+    if k == "lmhead":
+        hf, wte = rnd(M, C), rnd(V, C, scale=0.02)
+        tg = torch.from_numpy(rng.integers(0, V, size=M).astype(np.int32)).cuda()
+        logits = torch.empty(M, V, dtype=torch.float32, device="cuda")
+        loss = torch.empty(1, dtype=torch.float32, device="cuda")
+        ws = torch.empty(G.gpt2_op_lmhead_ce_workspace_bytes(G.GPT2_BF16, M, V), dtype=torch.uint8, device="cuda")
+        fn = lambda: G.gpt2_op_lmhead_ce(G.GPT2_BF16, hf, wte, tg, M, C, V, logits, None, loss, ws)
+        flops = lmhead_flops(WL, M)
+    elif k in ("c_attn", "attn_proj", "c_fc", "mlp_proj"):
+        N, K, epi = {"c_attn": (3 * C, C, 0), "attn_proj": (C, C, 2), "c_fc": (4 * C, C, 1),
+                     "mlp_proj": (C, 4 * C, 2)}[k]
+        A, W, b = rnd(M, K), rnd(N, K, scale=0.02), rnd(N, scale=0.01)
+        out = torch.zeros(M, N, dtype=torch.float32 if epi == 2 else bf, device="cuda")
+        fn = lambda: G.gpt2_op_linear(G.GPT2_BF16, epi, A, W, b, M, N, K, out)
+        flops = 2.0 * M * N * K
+    elif k == "attention":
+        qkv, y = rnd(M, 3 * C), torch.empty(M, C, dtype=bf, device="cuda")
+        fn = lambda: G.gpt2_op_attention(G.GPT2_BF16, qkv, WL.batch, WL.seq, H, C, y)
+        flops = WL.batch * 2.0 * C * WL.seq * (WL.seq + 1)
+    elif k == "layernorm":
+        x, g, b = rnd(M, C, dtype=torch.float32), rnd(C), rnd(C)
+        out = torch.empty(M, C, dtype=bf, device="cuda")
+        fn = lambda: G.gpt2_op_layernorm(G.GPT2_BF16, x, g, b, M, C, out)
+        flops = 0.0
+    else:
+        raise SystemExit(f"unknown kernel {k}")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"kernel": k, "ms_per_launch": ms, "tflops": flops / (ms / 1e3) / 1e12 if flops else None,
+                      "steps": args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", default=None,
+                    help="run one step alone: lmhead, c_attn, attn_proj, c_fc, mlp_proj, attention, layernorm")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.kernel:
+        run_kernel(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

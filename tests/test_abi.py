@@ -28,6 +28,7 @@ def test_binding_names_match_header():
     import transformer_decoder_lm_b200 as pkg
     for n in header_functions():
         assert callable(getattr(pkg.binding, n)), n
+        assert callable(getattr(pkg, n)), n         # re-exported by the package
 
 
 def test_workspace_bytes_and_config_checks():

@@ -9,7 +9,8 @@ from . import binding  # noqa: F401  (raises ImportError when libgpt2.so is miss
 from .binding import (  # noqa: F401
     GPT2_BF16, GPT2_FP32, GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID, GPT2Error,
     gpt2_workspace_bytes, gpt2_create, gpt2_forward, gpt2_loss, gpt2_forward_loss, gpt2_status,
-    gpt2_error_string, gpt2_destroy, gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear,
+    gpt2_error_string, gpt2_destroy, gpt2_launch_count, gpt2_set_timing_events, GPT2_TIMED_LMHEAD,
+    gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear,
     gpt2_op_attention, gpt2_op_lmhead_ce_workspace_bytes, gpt2_op_lmhead_ce, make_config,
 )
 from .model import GPT2Model, upload_weights  # noqa: F401

@@ -5,8 +5,8 @@
 // core modules in PyTorch", section 4.1 step 5: CrossEntropyLoss with its
 // mean reduction over the shifted targets).
 //
-// The lm_head epilogue left, per row and column tile, (m_i, s_i) with
-// s_i = sum over the tile of exp(z - m_i). Here one warp per row merges them:
+// The lm_head epilogue left, per row and column group, (m_i, s_i) with
+// s_i = sum over the group of exp(z - m_i). Here one warp per row merges them:
 // M = max m_i, S = sum s_i exp(m_i - M), lse = M + log S. A single block then
 // forms the mean in double precision in a fixed order (deterministic).
 #include "common.cuh"
@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256) ce_rows_kernel(const float2* __restrict__
   float m = -INFINITY, s = 0.f;
   for (int i = lane; i < n_tiles; i += 32) {
     const float2 p = part[(size_t)i * M + row];
+    if (p.x == -INFINITY) continue;   // a column group with no valid column
     const float mn = fmaxf(m, p.x);
     s = s * expf(m - mn) + p.y * expf(p.x - mn);
     m = mn;

@@ -7,30 +7,39 @@
 // with fp32 accumulation, A [M, K] and B [N, K] both K-major (the
 // nn.Linear [out, in] layout is already the K-major B operand).
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   warp 0      TMA producer: 128x64 A box and BNx64 B box per stage, 128-byte
-//               swizzle, STAGES-deep ring of shared-memory stages.
+//               swizzle, 4-deep ring of shared-memory stages.
 //   warp 1      allocates 2*BN TMEM columns and issues tcgen05.mma
 //               (M=128, N=BN, K=16, four per 64-wide k-block) into one of two
 //               TMEM accumulators; tcgen05.commit frees smem stages and hands
 //               finished accumulators to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, 32 columns at a
-//               time, fused bias / GELU(erf) / residual add / log-sum-exp.
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant (rows), each taking
+//               half of the tile's columns, 32 columns per tcgen05.ld:
+//                 EPI_BIAS / EPI_GELU  +bias (+GELU erf), bf16, staged in
+//                                      64B-swizzled smem, TMA store;
+//                 EPI_RESID            +bias, fp32, staged in 128B-swizzled
+//                                      smem, TMA reduce-add into the fp32
+//                                      residual stream (x += y without the SM
+//                                      ever reading x);
+//                 EPI_LMHEAD           online max / sum-exp per row over the
+//                                      valid columns, the target logit, and
+//                                      optionally the fp32 logits through an
+//                                      smem transposition (coalesced rows).
 // The double-buffered accumulator lets the epilogue of tile i overlap the
-// main loop of tile i+1. Tiles are walked M-fastest so that consecutive CTAs
-// share the B tile in L2 (the 77 MB wte of the lm_head is streamed ~once).
+// main loop of tile i+1. Tiles are walked M-fastest so that concurrently
+// running CTAs share B tiles in L2 (the 77 MB wte is streamed ~once).
 //
-// The lm_head epilogue never needs the logits in HBM: per row and column
-// tile it emits (max, sum exp(z - max)) and, in the tile holding the target
-// column, the target logit; a small kernel finishes the log-sum-exp.
-// Columns at or past N (the vocabulary padded up to the tile width by TMA
-// zero fill) are excluded from the sums and from the logits.
+// The lm_head epilogue never needs the logits in HBM: per row and half tile
+// it emits (max, sum exp(z - max)) and, where the target column lies, the
+// target logit; ce.cu finishes the log-sum-exp. Columns at or past N (the
+// vocabulary padded up to the tile width by TMA zero fill) are excluded from
+// the sums and from the logits.
 //
 // Every wait is bounded (common.cuh): on a timeout the kernel records
 // GPT2_ERR_DEVICE_TIMEOUT, lets its in-flight copies and MMAs land, frees its
 // TMEM and returns.
 #include <cudaTypedefs.h>
-
 #include <stdlib.h>
 
 #include <algorithm>
@@ -42,39 +51,56 @@ namespace g2 {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
-constexpr int TC_THREADS = 192;
-constexpr int STAGING_FLOATS = 4 * 32 * 33;   // per-warp 32x33 transposition buffers (lm_head logits)
+constexpr int TC_STAGES = 4;
+constexpr int TC_EPI_WARPS = 8;
+constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
+constexpr int STAGE_BUF_BYTES = 4096;   // per epilogue warp: 32 rows x 128 B
 
-template <int BN, int STAGES>
+template <int BN>
 struct TcLayout {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGING_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFFSET = STAGING_OFFSET + STAGING_FLOATS * 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
-  static constexpr int SMEM_BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + tmem holder, abort flag, align slack
-  static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
+  static constexpr int EPI_OFFSET = TC_STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFFSET = EPI_OFFSET + TC_EPI_WARPS * STAGE_BUF_BYTES;
+  static constexpr int NUM_BARS = 2 * TC_STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
+  static constexpr int SMEM_BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;   // + holders, 1 KB alignment slack
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
+  static constexpr int COLS_PER_WARP = BN / 2;
+  static constexpr int CHUNKS = COLS_PER_WARP / 32;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(COLS_PER_WARP % 32 == 0, "epilogue chunks are 32 columns");
 };
 
 __device__ __forceinline__ float bf2f(const bf16 v) { return __bfloat162float(v); }
 
-template <int BN, int STAGES, int EPI>
+// Bias slice of one 32-column chunk (bf16 -> fp32 registers); zeros past N.
+__device__ __forceinline__ void load_bias32(const bf16* bias, int col0, int N, float (&b)[32]) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int col = col0 + g * 8;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (col < N) w = __ldg(reinterpret_cast<const uint4*>(bias + col));
+    const bf16* bb = reinterpret_cast<const bf16*>(&w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[g * 8 + j] = bf2f(bb[j]);
+  }
+}
+
+template <int BN, int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs args) {
-  using L = TcLayout<BN, STAGES>;
+                   const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  using L = TcLayout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* empty = full + TC_STAGES;
+  uint64_t* tfull = empty + TC_STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* staging = reinterpret_cast<float*>(smem + L::STAGING_OFFSET);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -85,13 +111,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int nk = args.K / TC_BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < TC_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -100,6 +126,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI != EPI_LMHEAD) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, L::TMEM_COLS);
@@ -131,7 +158,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * TC_BK, n0);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == TC_STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -143,7 +170,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       // Let every issued copy land before the CTA can exit (bounded).
       volatile int no_abort = 0;
-      for (int s = 0; s < STAGES; ++s)
+      for (int s = 0; s < TC_STAGES; ++s)
         if (issued & (1u << s)) mbar_wait(&full[s], (issued_parity >> s) & 1u, &no_abort);
     }
   } else if (warp == 1) {
@@ -176,7 +203,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int k = 0; k < TC_BK / 16; ++k)
             mma_bf16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0);
           mma_commit(&empty[stage]);
-          if (++stage == STAGES) {
+          if (++stage == TC_STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -195,12 +222,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;   // TMEM lane quadrant this warp may access
-    float* stg = staging + q * (32 * 33);
+    const int q = warp & 3;                  // TMEM lane quadrant = rows q*32 .. q*32+31
+    const int half = (warp - 2) >> 2;        // which half of the tile's columns
+    uint8_t* sbuf = smem + L::EPI_OFFSET + (warp - 2) * STAGE_BUF_BYTES;
+    const uint32_t sb = smem_u32(sbuf);
+    constexpr float LOG2E = 1.4426950408889634f;
+    bool store_pending = false;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
+      const int row0 = m0 + q * 32;          // first row of this warp
+      const int row = row0 + lane;
+      const bool row_ok = row < M;
+      const int cbase = n0 + half * L::COLS_PER_WARP;
+
+      float run_max = -INFINITY, run_sum = 0.f, tgt_val = 0.f;
+      int tgt = -1;
+      if (EPI == EPI_LMHEAD) tgt = (row_ok && args.targets != nullptr) ? args.targets[row] : -1;
+
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
         if (lane == 0) {
           record_error(args.status, DEV_TIMEOUT);
@@ -209,20 +251,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
-      const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
-      const int row = m0 + q * 32 + lane;
-      const bool row_ok = row < M;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-
-      float run_max = -INFINITY, run_sum = 0.f, tgt_val = 0.f;
-      int tgt = -1;
-      if (EPI == EPI_LMHEAD) tgt = (row_ok && args.targets != nullptr) ? args.targets[row] : -1;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * L::COLS_PER_WARP;
 
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = n0 + c * 32;
+      for (int c = 0; c < L::CHUNKS; ++c) {
+        const int col0 = cbase + c * 32;
         if (col0 >= N) break;   // warp-uniform
+        float bias[32];
+        if (EPI != EPI_LMHEAD) load_bias32(static_cast<const bf16*>(args.bias), col0, N, bias);
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
         tmem_ld_wait();
@@ -231,45 +267,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 
         if (EPI == EPI_BIAS || EPI == EPI_GELU) {
-          const bf16* bias = static_cast<const bf16*>(args.bias);
-          bf16* o = static_cast<bf16*>(args.out) + (size_t)row * args.ldo + col0;
+          uint32_t pk[16];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = col0 + g * 8;
-            if (row_ok && col < N) {
-              const uint4 bw = *reinterpret_cast<const uint4*>(bias + col);
-              const bf16* bb = reinterpret_cast<const bf16*>(&bw);
-              float t[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                t[j] = v[g * 8 + j] + bf2f(bb[j]);
-                if (EPI == EPI_GELU) t[j] = gelu_erf(t[j]);
-              }
-              uint4 pk;
-              pk.x = pack_bf16x2(t[0], t[1]);
-              pk.y = pack_bf16x2(t[2], t[3]);
-              pk.z = pack_bf16x2(t[4], t[5]);
-              pk.w = pack_bf16x2(t[6], t[7]);
-              *reinterpret_cast<uint4*>(o + g * 8) = pk;
+          for (int j = 0; j < 16; ++j) {
+            float a = v[2 * j] + bias[2 * j], b = v[2 * j + 1] + bias[2 * j + 1];
+            if (EPI == EPI_GELU) {
+              a = gelu_erf(a);
+              b = gelu_erf(b);
             }
+            pk[j] = pack_bf16x2(a, b);
           }
+          if (store_pending) {       // the previous chunk's TMA store must have read the buffer
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
+          // 32 rows x 64 B, 64-byte swizzle: 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(sb + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                         pk[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M) {
+            tma_store_2d(&tmC, sbuf, col0, row0);
+            bulk_commit();
+          }
+          store_pending = true;
         } else if (EPI == EPI_RESID) {
-          const bf16* bias = static_cast<const bf16*>(args.bias);
-          float* o = static_cast<float*>(args.out) + (size_t)row * args.ldo + col0;
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const int col = col0 + g * 4;
-            if (row_ok && col < N) {
-              const uint2 bw = *reinterpret_cast<const uint2*>(bias + col);
-              const bf16* bb = reinterpret_cast<const bf16*>(&bw);
-              float4 x = *reinterpret_cast<float4*>(o + g * 4);
-              x.x += v[g * 4 + 0] + bf2f(bb[0]);
-              x.y += v[g * 4 + 1] + bf2f(bb[1]);
-              x.z += v[g * 4 + 2] + bf2f(bb[2]);
-              x.w += v[g * 4 + 3] + bf2f(bb[3]);
-              *reinterpret_cast<float4*>(o + g * 4) = x;
-            }
+          for (int j = 0; j < 32; ++j) v[j] += bias[j];
+          if (store_pending) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
           }
+          // 32 rows x 128 B, 128-byte swizzle: unit j of row r at unit j ^ (r & 7)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(sb + lane * 128 + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]),
+                         __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M) {
+            tma_reduce_add_2d(&tmC, sbuf, col0, row0);
+            bulk_commit();
+          }
+          store_pending = true;
         } else {  // EPI_LMHEAD
           const int nvalid = min(32, N - col0);
           float cmax = -INFINITY;
@@ -277,29 +319,40 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int j = 0; j < 32; ++j)
             if (j < nvalid) cmax = fmaxf(cmax, v[j]);
           const float new_max = fmaxf(run_max, cmax);
-          constexpr float LOG2E = 1.4426950408889634f;
           const float nm2 = new_max * LOG2E;
-          float s = run_sum * exp2f(run_max * LOG2E - nm2);
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j < nvalid) s += exp2f(fmaf(v[j], LOG2E, -nm2));
-            if (col0 + j == tgt) tgt_val = v[j];
+          for (int j = 0; j < 32; j += 4) {
+            if (j + 0 < nvalid) s0 += exp2f(fmaf(v[j + 0], LOG2E, -nm2));
+            if (j + 1 < nvalid) s1 += exp2f(fmaf(v[j + 1], LOG2E, -nm2));
+            if (j + 2 < nvalid) s2 += exp2f(fmaf(v[j + 2], LOG2E, -nm2));
+            if (j + 3 < nvalid) s3 += exp2f(fmaf(v[j + 3], LOG2E, -nm2));
           }
-          run_sum = s;
+          run_sum = run_sum * exp2f(run_max * LOG2E - nm2) + ((s0 + s1) + (s2 + s3));
           run_max = new_max;
-          if (args.out != nullptr) {
-            // Transpose through shared memory so that each row segment is
-            // written by 32 consecutive lanes (the logits row pitch V is odd,
-            // so rows are only 4-byte aligned).
+          const int tj = tgt - col0;
+          if (tj >= 0 && tj < 32) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = v[j];
+            for (int j = 0; j < 32; ++j)
+              if (j == tj) tgt_val = v[j];
+          }
+          if (args.out != nullptr) {
+            // Transpose through shared memory (128-byte swizzled rows) so that
+            // each logits row segment is written by 32 consecutive lanes: the
+            // logits row pitch V is odd, so rows are only 4-byte aligned.
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(sb + lane * 128 + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]),
+                           __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
+                           __float_as_uint(v[4 * j + 3]));
             __syncwarp();
             float* lg = static_cast<float*>(args.out);
             const int gcol = col0 + lane;
-#pragma unroll 4
+            const bool col_ok = gcol < N;
+#pragma unroll 8
             for (int rr = 0; rr < 32; ++rr) {
-              const int grow = m0 + q * 32 + rr;
-              if (grow < M && gcol < N) lg[(size_t)grow * args.ldo + gcol] = stg[rr * 33 + lane];
+              const float val = ld_shared_f32(sb + rr * 128 + (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+              if (row0 + rr < M && col_ok) lg[(size_t)(row0 + rr) * args.ldo + gcol] = val;
             }
             __syncwarp();
           }
@@ -311,10 +364,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0) mbar_arrive(&tempty[acc]);
 
       if (EPI == EPI_LMHEAD && row_ok) {
-        args.part[(size_t)n_blk * M + row] = make_float2(run_max, run_sum);
-        if (tgt >= n0 && tgt < n0 + BN && tgt < N) args.tgt_logit[row] = tgt_val;
+        // one partial per (row, half tile): rows of `part` are column groups of BN/2
+        args.part[(size_t)(n_blk * 2 + half) * M + row] = make_float2(run_max, run_sum);
+        if (tgt >= cbase && tgt < cbase + L::COLS_PER_WARP && tgt < N) args.tgt_logit[row] = tgt_val;
       }
     }
+    if (EPI != EPI_LMHEAD && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   __syncthreads();
@@ -340,38 +396,44 @@ bool load_encode() {
   return true;
 }
 
-template <int BN>
-constexpr int stages_for() {
-  return BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* base, uint64_t rows, uint64_t cols,
+               uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  if (!load_encode()) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * esize) & 15) || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * (uint64_t)esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 template <int BN, int EPI>
-cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& a, int num_sms,
-                       cudaStream_t s) {
-  constexpr int ST = stages_for<BN>();
-  using L = TcLayout<BN, ST>;
+cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC, const GemmArgs& a,
+                       int num_sms, cudaStream_t s) {
+  using L = TcLayout<BN>;
   const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
   const int grid = std::min(tiles, num_sms);
   if (grid <= 0) return cudaSuccess;
-  gemm_tc_kernel<BN, ST, EPI><<<grid, TC_THREADS, L::SMEM_BYTES, s>>>(tA, tB, a);
+  gemm_tc_kernel<BN, EPI><<<grid, TC_THREADS, L::SMEM_BYTES, s>>>(tA, tB, tC, a);
   return cudaGetLastError();
 }
 
 template <int BN, int EPI>
 cudaError_t set_attr_one() {
-  constexpr int ST = stages_for<BN>();
-  return cudaFuncSetAttribute(gemm_tc_kernel<BN, ST, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcLayout<BN, ST>::SMEM_BYTES);
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcLayout<BN>::SMEM_BYTES);
 }
 
 template <int BN>
-cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& a, int num_sms,
-                      cudaStream_t s) {
+cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
+                      const GemmArgs& a, int num_sms, cudaStream_t s) {
   switch (epi) {
-    case EPI_BIAS: return launch_one<BN, EPI_BIAS>(tA, tB, a, num_sms, s);
-    case EPI_GELU: return launch_one<BN, EPI_GELU>(tA, tB, a, num_sms, s);
-    case EPI_RESID: return launch_one<BN, EPI_RESID>(tA, tB, a, num_sms, s);
-    case EPI_LMHEAD: return launch_one<BN, EPI_LMHEAD>(tA, tB, a, num_sms, s);
+    case EPI_BIAS: return launch_one<BN, EPI_BIAS>(tA, tB, tC, a, num_sms, s);
+    case EPI_GELU: return launch_one<BN, EPI_GELU>(tA, tB, tC, a, num_sms, s);
+    case EPI_RESID: return launch_one<BN, EPI_RESID>(tA, tB, tC, a, num_sms, s);
+    case EPI_LMHEAD: return launch_one<BN, EPI_LMHEAD>(tA, tB, tC, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -379,19 +441,19 @@ cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, con
 
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                     uint32_t box_rows) {
-  if (!load_encode()) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15) || rows == 0 || cols == 0) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, ld, 64, box_rows,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int gemm_tc_n_tiles(int N, int bn) { return (N + bn - 1) / bn; }
+bool make_tmap_out_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+  return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+bool make_tmap_out_f32(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+  return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int gemm_tc_n_tiles(int N, int bn) { return 2 * ((N + bn - 1) / bn); }
 
 int gemm_tc_pick_bn(int M, int N, int num_sms) {
   // G2_GEMM_BN=64|128|256 pins the tile width (tests use it to cover every
@@ -400,10 +462,11 @@ int gemm_tc_pick_bn(int M, int N, int num_sms) {
     const int v = atoi(e);
     if (v == 64 || v == 128 || v == 256) return v;
   }
-  // Estimated cost = waves x per-tile cost. Narrow tiles re-read A from shared
-  // memory more often per FLOP, so their per-column cost is higher.
+  // Estimated cost = waves x per-tile cost. Narrower tiles re-read A from
+  // shared memory more often per FLOP (the 128-row MMA at N=128 runs at
+  // about 60% of the N=256 rate), so their per-column cost is higher.
   const int cand[3] = {256, 128, 64};
-  const double unit[3] = {256.0, 136.0, 96.0};
+  const double unit[3] = {256.0, 200.0, 150.0};
   const int mt = (M + TC_BM - 1) / TC_BM;
   int best = 256;
   double best_cost = 1e30;
@@ -419,12 +482,12 @@ int gemm_tc_pick_bn(int M, int N, int num_sms) {
   return best;
 }
 
-cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& a,
-                           int num_sms, cudaStream_t s) {
+cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
+                           const GemmArgs& a, int num_sms, cudaStream_t s) {
   switch (bn) {
-    case 256: return launch_bn<256>(epi, tA, tB, a, num_sms, s);
-    case 128: return launch_bn<128>(epi, tA, tB, a, num_sms, s);
-    case 64: return launch_bn<64>(epi, tA, tB, a, num_sms, s);
+    case 256: return launch_bn<256>(epi, tA, tB, tC, a, num_sms, s);
+    case 128: return launch_bn<128>(epi, tA, tB, tC, a, num_sms, s);
+    case 64: return launch_bn<64>(epi, tA, tB, tC, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

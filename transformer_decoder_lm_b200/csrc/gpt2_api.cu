@@ -17,6 +17,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -34,6 +35,10 @@ inline int bn_index(int bn) { return bn == 256 ? 0 : (bn == 128 ? 1 : 2); }
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// lm_head partials per row: two column groups per tile of width >= 128 (tcgen05
+// path) or one per 64-column tile (SIMT path); both fit in 2 * ceil(V / 128).
+inline size_t lmhead_groups(int V) { return 2 * (size_t)((V + LMHEAD_MIN_BN - 1) / LMHEAD_MIN_BN); }
+
 struct LayerPtrs {
   const void *ln1_g, *ln1_b, *attn_w, *attn_b, *attn_proj_w, *attn_proj_b;
   const void *ln2_g, *ln2_b, *fc_w, *fc_b, *mlp_proj_w, *mlp_proj_b;
@@ -50,7 +55,7 @@ struct Plan {
 Plan plan_workspace(const gpt2_config_t& c, long M) {
   const size_t es = c.dtype == GPT2_BF16 ? 2 : 4;
   const size_t C = (size_t)c.n_embd;
-  const size_t n_tiles = (size_t)((c.vocab + 63) / 64);   // the narrowest lm_head tile width
+  const size_t n_tiles = lmhead_groups(c.vocab);
   Plan p;
   size_t o = 0;
   p.x = o;      o += align256(M * C * 4);
@@ -134,7 +139,7 @@ namespace {
 
 // One Linear layer of the schedule.
 int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, const void* W, const CUtensorMap* wmaps,
-               const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s) {
+               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s) {
   GemmArgs a{};
   a.M = M;
   a.N = N;
@@ -146,7 +151,7 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   cudaError_t e;
   if (m->bf16) {
     const int bn = gemm_tc_pick_bn(M, N, m->num_sms);
-    e = gemm_tc_launch(epi, bn, *tmA, wmaps[bn_index(bn)], a, m->num_sms, s);
+    e = gemm_tc_launch(epi, bn, *tmA, wmaps[bn_index(bn)], *tmC, a, m->num_sms, s);
   } else {
     e = gemm_simt_launch(epi, static_cast<const float*>(A), static_cast<const float*>(W), a, s);
   }
@@ -164,10 +169,12 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
 
   const gpt2_config_t& c = m->cfg;
   const int M = B * T, C = c.n_embd, H = c.n_head, V = c.vocab;
-  CUtensorMap tm_h, tm_y, tm_f;
+  CUtensorMap tm_h, tm_y, tm_f, out_qkv, out_f, out_x;
   if (m->bf16) {
     if (!make_tmap_bf16(&tm_h, m->h, M, C, C, 128) || !make_tmap_bf16(&tm_y, m->y, M, C, C, 128) ||
-        !make_tmap_bf16(&tm_f, m->f, M, 4 * C, 4 * C, 128))
+        !make_tmap_bf16(&tm_f, m->f, M, 4 * C, 4 * C, 128) ||
+        !make_tmap_out_bf16(&out_qkv, m->qkv, M, 3 * C, 3 * C) || !make_tmap_out_bf16(&out_f, m->f, M, 4 * C, 4 * C) ||
+        !make_tmap_out_f32(&out_x, m->x, M, C, C))
       return GPT2_ERR_CUDA;
   }
   int rc = GPT2_OK;
@@ -187,12 +194,12 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     const LayerPtrs& L = m->layers[l];
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
-    G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, L.attn_b, M, 3 * C, C, m->qkv, 3 * C, s));
+    G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C, m->qkv, 3 * C, s));
     G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, m->status, s));
-    G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, L.attn_proj_b, M, C, C, m->x, C, s));
+    G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
-    G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, L.fc_b, M, 4 * C, C, m->f, 4 * C, s));
-    G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, L.mlp_proj_b, M, C, 4 * C, m->x, C, s));
+    G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, &out_f, L.fc_b, M, 4 * C, C, m->f, 4 * C, s));
+    G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C, s));
     m->launches += 7;
   }
   G2_CK(layernorm_launch(m->bf16, m->x, m->lnf_g, m->lnf_b, m->h, M, C, s));
@@ -213,9 +220,9 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     int n_tiles;
     if (m->ev_lm_begin) G2_CK(cudaEventRecord(m->ev_lm_begin, s));
     if (m->bf16) {
-      const int bn = gemm_tc_pick_bn(M, V, m->num_sms);
+      const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms), LMHEAD_MIN_BN);
       n_tiles = gemm_tc_n_tiles(V, bn);
-      G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, tm_h, m->wte_map[bn_index(bn)], a, m->num_sms, s));
+      G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, tm_h, m->wte_map[bn_index(bn)], tm_h, a, m->num_sms, s));
     } else {
       n_tiles = (V + SIMT_BN - 1) / SIMT_BN;
       G2_CK(gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(m->h), static_cast<const float*>(m->wte), a, s));
@@ -441,9 +448,12 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
   int rc = device_setup(nullptr, &sms);
   if (rc != GPT2_OK) return rc;
   const int bn = gemm_tc_pick_bn(M, N, sms);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!make_tmap_bf16(&ta, A, M, K, K, 128) || !make_tmap_bf16(&tb, W, N, K, K, bn)) return GPT2_ERR_CUDA;
-  return gemm_tc_launch(epilogue, bn, ta, tb, a, sms, s) == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+  const bool ok_c = epilogue == GPT2_EPI_BIAS_RESID ? make_tmap_out_f32(&tc, out, M, N, N)
+                                                     : make_tmap_out_bf16(&tc, out, M, N, N);
+  if (!ok_c) return GPT2_ERR_CUDA;
+  return gemm_tc_launch(epilogue, bn, ta, tb, tc, a, sms, s) == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
 int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, void* y, int* status, void* stream) {
@@ -460,8 +470,7 @@ int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, vo
 
 size_t gpt2_op_lmhead_ce_workspace_bytes(int dtype, int M, int V) {
   if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || M < 1 || V < 1) return 0;
-  const size_t n_tiles = (size_t)((V + 63) / 64);
-  return align256(n_tiles * (size_t)M * sizeof(float2)) + 2 * align256((size_t)M * 4);
+  return align256(lmhead_groups(V) * (size_t)M * sizeof(float2)) + 2 * align256((size_t)M * 4);
 }
 
 int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t* targets, int M, int C, int V,
@@ -473,7 +482,7 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
   if (ws_bytes < gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V)) return GPT2_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t n_tiles_max = (size_t)((V + 63) / 64);
+  const size_t n_tiles_max = lmhead_groups(V);
   float2* part = reinterpret_cast<float2*>(ws);
   float* tgt = reinterpret_cast<float*>(ws + align256(n_tiles_max * (size_t)M * sizeof(float2)));
   float* tok = tgt + align256((size_t)M * 4) / 4;
@@ -493,11 +502,11 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
     int sms = 0;
     int rc = device_setup(nullptr, &sms);
     if (rc != GPT2_OK) return rc;
-    const int bn = gemm_tc_pick_bn(M, V, sms);
+    const int bn = std::max(gemm_tc_pick_bn(M, V, sms), LMHEAD_MIN_BN);
     n_tiles = gemm_tc_n_tiles(V, bn);
     CUtensorMap ta, tb;
     if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;
-    if (gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, a, sms, s) != cudaSuccess) return GPT2_ERR_CUDA;
+    if (gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, ta, a, sms, s) != cudaSuccess) return GPT2_ERR_CUDA;
   } else {
     n_tiles = (V + SIMT_BN - 1) / SIMT_BN;
     if (gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(hf), static_cast<const float*>(wte), a, s) !=

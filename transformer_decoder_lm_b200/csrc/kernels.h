@@ -18,25 +18,33 @@ struct GemmArgs {
                            // EPI_LMHEAD: fp32 logits [M, ldo] or NULL
   long long ldo;
   const int* targets;      // EPI_LMHEAD: [M]
-  float2* part;            // EPI_LMHEAD: per (column tile, row) (max, sum exp(z - max)), [n_tiles, M]
+  float2* part;            // EPI_LMHEAD: per (column group, row) (max, sum exp(z - max)), [n_groups, M]
   float* tgt_logit;        // EPI_LMHEAD: [M] logit of the target column
   int* status;
 };
 
 // ---- tensor maps (host) -------------------------------------------------
-// Encode a 2-D bf16 row-major tensor [rows, cols] (row pitch `ld` elements)
-// read in boxes of box_rows x 64 columns with 128-byte swizzling.
+// GEMM operand: a 2-D bf16 row-major tensor [rows, cols] (row pitch `ld`
+// elements) read in boxes of box_rows x 64 columns with 128-byte swizzling.
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                     uint32_t box_rows);
+// GEMM outputs written by the epilogue in 32 x 32 boxes: bf16 (64-byte
+// swizzle, TMA store) and fp32 (128-byte swizzle, TMA reduce-add).
+bool make_tmap_out_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
+bool make_tmap_out_f32(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
+// Column groups of lm_head partials for N columns (two per tile of width bn).
+int gemm_tc_n_tiles(int N, int bn);
+// The lm_head runs with tiles of at least this width.
+constexpr int LMHEAD_MIN_BN = 128;
 
 // ---- tcgen05 GEMM (bf16) -------------------------------------------------
 // C = A[M,K] . B[N,K]^T with the epilogue `epi`. K % 64 == 0, N % 8 == 0.
-// tmA: box 128 x 64 over A; tmB: box BN x 64 over B, BN from gemm_tc_pick_bn.
+// tmA: box 128 x 64 over A; tmB: box BN x 64 over B, BN from gemm_tc_pick_bn;
+// tmC: the output map (make_tmap_out_*; unused by EPI_LMHEAD).
 int gemm_tc_pick_bn(int M, int N, int num_sms);
-cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tmA, const CUtensorMap& tmB,
+cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
                            const GemmArgs& a, int num_sms, cudaStream_t s);
 cudaError_t gemm_tc_set_attributes();
-int gemm_tc_n_tiles(int N, int bn);
 
 // ---- SIMT fp32 GEMM (fp32 mode) ------------------------------------------
 constexpr int SIMT_BN = 64;
