@@ -251,6 +251,7 @@ cudaError_t attention_launch(bool bf16_, const void* qkv, void* y, int B, int T,
   const int D = C / H;
   if (bf16_) {
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    if (D == 64) return attention_tc_launch(qkv, y, B, T, H, C, status, s);
     dim3 grid((T + 63) / 64, H, B);
     if (D == 64)
       attn_fwd_bf16_kernel<64><<<grid, 128, 0, s>>>(static_cast<const bf16*>(qkv), static_cast<bf16*>(y), T, H, C,

@@ -1,0 +1,333 @@
+// attention_tc.cu - causal flash attention on tcgen05 / TMEM / TMA (sm_100a, d_head 64).
+//
+// Per sequence b, head h and 128-query tile: y = softmax(q k^T / sqrt(D),
+// -inf where key j > query i) v ("Reproducing GPT-2 124M", sections 2.1-2.2;
+// "Hand-writing GPT-2 from scratch: the Transformer decoder core modules in
+// PyTorch", section 3.3: key j is visible iff j <= i), online over 128-key
+// tiles so the T x T score matrix never exists.
+//
+// One CTA per (b, h, query tile), 6 warps, two CTAs per SM:
+//   warp 0     TMA: the 128x64 Q box once, then K and V boxes of 128 keys x 64
+//              into a 2-deep ring, all read in place from the c_attn output
+//              through a 3-D map [B, T, 3C] (rows past T read as zero).
+//   warp 1     tcgen05.mma: S = Q K^T (M=128, N=128, K=64) into TMEM, then
+//              O += P V (M=128, N=64, K=128; V used MN-major straight from the
+//              TMA box) into a TMEM accumulator. S of tile j+1 is issued while
+//              the softmax warps work on tile j.
+//   warps 2-5  one thread per query row: read the S row from TMEM, scale by
+//              log2(e)/sqrt(D), mask the diagonal tile, keep the running max m
+//              and sum l in registers, write P = exp2(s - m) as bf16 into
+//              128B-swizzled smem (the A operand of the PV product). The max
+//              used for P is raised only when the row max grows by more than
+//              2^8; then the O row in TMEM is rescaled first (tcgen05.ld / st).
+//              At the end O / l goes out through smem and a 3-D TMA store
+//              (rows past T are not written).
+// Key tiles above the diagonal are never loaded or multiplied. Query tiles
+// are scheduled longest first.
+//
+// Every wait is bounded (common.cuh); on a timeout the CTA records
+// GPT2_ERR_DEVICE_TIMEOUT, drains its copies and MMAs, frees TMEM and exits.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace g2 {
+
+namespace {
+constexpr int AT_BQ = 128, AT_BK = 128, AT_D = 64;
+constexpr int AT_THREADS = 192;
+constexpr int TILE_BYTES = 128 * 64 * 2;                 // one 128 x 64 bf16 box
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + TILE_BYTES;                // 2 stages
+constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;            // 2 stages
+constexpr int OFF_P = OFF_V + 2 * TILE_BYTES;            // 128 x 128 bf16 = two 64-key sub-tiles
+constexpr int OFF_BAR = OFF_P + 2 * TILE_BYTES;
+constexpr int NUM_BARS = 11;
+constexpr int AT_SMEM = OFF_BAR + NUM_BARS * 8 + 8;
+constexpr uint32_t TMEM_COLS = 256;                      // S: cols [0,128), O: cols [128,192)
+constexpr uint32_t TM_S = 0, TM_O = 128;
+constexpr float RESCALE_THRESHOLD = 8.0f;                // log2 units
+}  // namespace
+
+__global__ void __launch_bounds__(AT_THREADS, 2)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_y, int B,
+                       int T, int H, int C, float scale_log2, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_free = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* pv_done = bars + 8;
+  uint64_t* drain = bars + 9;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int QT = (T + AT_BQ - 1) / AT_BQ;
+  const int BH = B * H;
+  const int qt = QT - 1 - (int)(blockIdx.x / BH);   // longest query tiles first
+  const int bh = blockIdx.x % BH;
+  const int b = bh / H, h = bh % H;
+  const int q0 = qt * AT_BQ;
+  const int n_kv = qt + 1;
+
+  if ((smem_u32(smem) & 1023u) != 0) {   // the swizzled TMA boxes need 1 KB alignment
+    if (threadIdx.x == 0) record_error(status, DEV_TIMEOUT);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], (i == 6 || i == 7) ? 4 : 1);   // s_free, p_full: 4 warps
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_y);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t issued = 0, issued_parity = 0;
+      mbar_arrive_expect_tx(q_full, TILE_BYTES);
+      tma_load_3d(smem + OFF_Q, &tm_qkv, q_full, h * AT_D, q0, b);
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE_BYTES);
+        tma_load_3d(smem + OFF_K + st * TILE_BYTES, &tm_qkv, &kv_full[st], C + h * AT_D, j * AT_BK, b);
+        tma_load_3d(smem + OFF_V + st * TILE_BYTES, &tm_qkv, &kv_full[st], 2 * C + h * AT_D, j * AT_BK, b);
+        issued |= 1u << st;
+        issued_parity = (issued_parity & ~(1u << st)) | (ph << st);
+      }
+      if (!ok) {
+        record_error(status, DEV_TIMEOUT);
+        *abort_flag = 1;
+      }
+      volatile int no_abort = 0;
+      mbar_wait(q_full, 0, &no_abort);
+      for (int st = 0; st < 2; ++st)
+        if (issued & (1u << st)) mbar_wait(&kv_full[st], (issued_parity >> st) & 1u, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(AT_BQ, AT_BK);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32_bmn(AT_BQ, AT_D);
+      const uint32_t tS = tmem_base + TM_S, tO = tmem_base + TM_O;
+      const uint64_t qdesc = sdesc_kmajor_sw128(smem_u32(smem + OFF_Q));
+      const uint32_t p_addr = smem_u32(smem + OFF_P);
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        const uint64_t kdesc = sdesc_kmajor_sw128(smem_u32(smem + OFF_K));
+#pragma unroll
+        for (int k = 0; k < AT_D / 16; ++k) mma_bf16_ss(tS, qdesc + 2 * k, kdesc + 2 * k, IDESC_S, k > 0);
+        mma_commit(s_full);
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv) {   // S of the next tile, overlapping the softmax of this one
+          const int st = (j + 1) & 1;
+          if (!mbar_wait(&kv_full[st], ((j + 1) >> 1) & 1, abort_flag) || !mbar_wait(s_free, j & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kdesc = sdesc_kmajor_sw128(smem_u32(smem + OFF_K + st * TILE_BYTES));
+#pragma unroll
+          for (int k = 0; k < AT_D / 16; ++k) mma_bf16_ss(tS, qdesc + 2 * k, kdesc + 2 * k, IDESC_S, k > 0);
+          mma_commit(s_full);
+        }
+        if (!mbar_wait(p_full, j & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + OFF_V + (j & 1) * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < AT_BK / 16; ++k) {
+          // P: K-major, keys 16k..16k+15 live in 64-key sub-tile k/4 at byte 32*(k%4)
+          const uint64_t pdesc = sdesc_kmajor_sw128(p_addr + (k >> 2) * TILE_BYTES) + 2 * (k & 3);
+          // V: MN-major, 16 key rows per step = 2048 B
+          const uint64_t vdesc = sdesc_mnmajor_sw128(v_addr + k * 2048);
+          mma_bf16_ss(tO, pdesc, vdesc, IDESC_O, (j | k) != 0);
+        }
+        mma_commit(&kv_empty[j & 1]);
+        mma_commit(pv_done);
+      }
+      if (!ok) {
+        record_error(status, DEV_TIMEOUT);
+        *abort_flag = 1;
+      }
+      mma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else {
+    // ----------------------------------------------------- softmax / output
+    const int qd = warp & 3;                     // TMEM lane quadrant
+    const int r = qd * 32 + lane;                // row within the tile
+    const int i = q0 + r;                        // query position in the sequence
+    const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
+    const uint32_t tS = tmem_base + TM_S + lane_off, tO = tmem_base + TM_O + lane_off;
+    const uint32_t p_addr = smem_u32(smem + OFF_P);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait(s_full, j & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld_32x32b_x32(tS + c * 32, rr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+
+      const int key0 = j * AT_BK;
+      const bool diag = (j == qt);
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 128; ++e) {
+        float v = s[e] * scale_log2;
+        if (diag && (key0 + e > i || key0 + e >= T)) v = -INFINITY;
+        s[e] = v;
+        tmax = fmaxf(tmax, v);
+      }
+      const float m_new = fmaxf(m, tmax);
+      const bool raise = m_new > m + RESCALE_THRESHOLD;
+      float alpha = 1.f;
+      if (raise) {
+        alpha = exp2f(m - m_new);   // 0 on the first tile (m = -inf)
+        m = m_new;
+      }
+      l *= alpha;
+      uint32_t pk[64];
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float p0 = exp2f(s[2 * e] - m), p1 = exp2f(s[2 * e + 1] - m);
+        ls0 += p0;
+        ls1 += p1;
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      l += ls0 + ls1;
+
+      if (j > 0) {   // PV of the previous tile done: O is stable and the P buffer is free
+        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st_32x32b_x32(tO + c * 32, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      // P row r: 256 B as 16 units of 16 B; unit u in sub-tile u/8 at swizzled slot (u%8) ^ (r%8)
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        st_shared_v4(p_addr + (u >> 3) * TILE_BYTES + r * 128 + (((u & 7) ^ (r & 7)) << 4), pk[4 * u],
+                     pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + c * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[c * 16 + e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+      }
+      // stage 32 rows x 128 B (128-byte swizzle) in this warp's slice of the P buffer, then TMA store
+      uint8_t* stg = smem + OFF_P + qd * 4096;
+      const uint32_t sb = smem_u32(stg);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(sb + lane * 128 + ((u ^ (lane & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
+                     pk[4 * u + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && q0 + qd * 32 < T) {
+        tma_store_3d(&tm_y, stg, h * AT_D, q0 + qd * 32, b);
+        bulk_commit();
+        bulk_wait_all();
+      }
+      __syncwarp();
+    } else if (lane == 0) {
+      record_error(status, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, int* status, cudaStream_t s) {
+  if (B <= 0 || T <= 0) return cudaSuccess;
+  if (C / H != AT_D) return cudaErrorInvalidValue;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tq, ty;
+  // qkv as [B][T][3C], boxes of 64 columns x 128 rows; y as [B][T][C], boxes of 64 x 32.
+  if (!make_tmap_3d_bf16(&tq, qkv, 3 * (uint64_t)C, T, B, 3 * (uint64_t)C, (uint64_t)T * 3 * C, 64, 128) ||
+      !make_tmap_3d_bf16(&ty, y, C, T, B, C, (uint64_t)T * C, 64, 32))
+    return cudaErrorInvalidValue;
+  const int QT = (T + AT_BQ - 1) / AT_BQ;
+  const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)AT_D));
+  attn_fwd_tc_kernel<<<B * H * QT, AT_THREADS, AT_SMEM, s>>>(tq, ty, B, T, H, C, scale_log2, status);
+  return cudaGetLastError();
+}
+
+}  // namespace g2

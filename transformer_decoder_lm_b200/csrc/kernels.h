@@ -32,6 +32,10 @@ bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
 // swizzle, TMA store) and fp32 (128-byte swizzle, TMA reduce-add).
 bool make_tmap_out_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
 bool make_tmap_out_f32(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
+// A 3-D bf16 tensor [d2][d1][d0] (row strides s1, s2 in elements) read or
+// written in boxes of box1 rows x box0 (= 64) columns, 128-byte swizzle.
+bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                       uint64_t s2, uint32_t box0, uint32_t box1);
 // Column groups of lm_head partials for N columns (two per tile of width bn).
 int gemm_tc_n_tiles(int N, int bn);
 // The lm_head runs with tiles of at least this width.
@@ -57,6 +61,8 @@ cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const voi
                              cudaStream_t s);
 
 // ---- attention ---------------------------------------------------------------
+// tcgen05 flash attention (bf16, d_head 64); attention_launch dispatches to it.
+cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, int* status, cudaStream_t s);
 cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C, int* status,
                              cudaStream_t s);
 
