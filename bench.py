@@ -328,10 +328,10 @@ def run_kernel(args):
         return (torch.from_numpy(rng.standard_normal(shape).astype(np.float32)) * scale).to("cuda", dtype)
 
     k = args.kernel
-    if k == "lmhead":
+    if k in ("lmhead", "lmhead_ce"):
         hf, wte = rnd(M, C), rnd(V, C, scale=0.02)
         tg = torch.from_numpy(rng.integers(0, V, size=M).astype(np.int32)).cuda()
-        logits = torch.empty(M, V, dtype=torch.float32, device="cuda")
+        logits = torch.empty(M, V, dtype=torch.float32, device="cuda") if k == "lmhead" else None
         loss = torch.empty(1, dtype=torch.float32, device="cuda")
         ws = torch.empty(G.gpt2_op_lmhead_ce_workspace_bytes(G.GPT2_BF16, M, V), dtype=torch.uint8, device="cuda")
         fn = lambda: G.gpt2_op_lmhead_ce(G.GPT2_BF16, hf, wte, tg, M, C, V, logits, None, loss, ws)
@@ -371,7 +371,8 @@ def run_kernel(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None,
-                    help="run one step alone: lmhead, c_attn, attn_proj, c_fc, mlp_proj, attention, layernorm")
+                    help="run one step alone: lmhead, lmhead_ce (no logits), c_attn, attn_proj, c_fc, mlp_proj, "
+                         "attention, layernorm")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)

@@ -128,6 +128,29 @@ def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
         assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-4)
 
 
+def test_gelu_epilogue_within_one_bf16_ulp(G):
+    """The c_fc epilogue's GELU on exactly representable pre-activations in
+    [-8, 8] (identity weights, zero bias) against the fp64 erf form, after the
+    same bf16 rounding: at most one bf16 ulp apart (the erf approximation's
+    error, a few 1e-7 absolute, only matters at rounding boundaries)."""
+    M = N = K = 64 * 4
+    xs = synthetic.round_to_bf16(np.linspace(-8, 8, M).astype(np.float32))
+    A = np.zeros((M, K), np.float32)
+    A[np.arange(M), np.arange(M) % K] = xs
+    W = np.eye(N, K, dtype=np.float32)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    G.gpt2_op_linear(G.GPT2_BF16, 1, dev(A, "bf16"), dev(W, "bf16"), dev(np.zeros(N, np.float32), "bf16"), M, N, K,
+                     out)
+    got = out.float().cpu().numpy()[np.arange(M), np.arange(M) % K]
+    exact = O.gelu(xs.astype(np.float64))
+    ref = torch.from_numpy(exact).to(torch.bfloat16).float().numpy()
+    # one bf16 ulp, plus 1e-6 absolute: for x < -5 the exact value is below
+    # 1e-6 and fp32's 1 + erf(x / sqrt 2) cancels to 0 (as CUDA's erff does)
+    ulp = np.abs(ref) * 2.0 ** -7
+    assert np.all(np.abs(got - ref) <= ulp + 1e-6)
+    assert np.abs(got - exact).max() <= 2.0 ** -8 * 8
+
+
 @pytest.mark.parametrize("epi", [0, 1, 2])
 def test_linear_fp32_simt(G, epi):
     M, N, K = 130, 200, 72

@@ -196,46 +196,48 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         break;
       }
       tc_fence_after();
-      float s[128];
+      // the whole S row: four TMEM loads, one wait, then release S to the MMA warp
+      uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(tS + c * 32, rr);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, sr[c]);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
 
       const int key0 = j * AT_BK;
-      const bool diag = (j == qt);
+      if (j == qt) {   // diagonal tile: keys after the query (or past T) get -inf
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (key0 + c * 32 + e > i || key0 + c * 32 + e >= T) sr[c][e] = __float_as_uint(-INFINITY);
+      }
       float tmax = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        float v = s[e] * scale_log2;
-        if (diag && (key0 + e > i || key0 + e >= T)) v = -INFINITY;
-        s[e] = v;
-        tmax = fmaxf(tmax, v);
-      }
-      const float m_new = fmaxf(m, tmax);
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(sr[c][e]));
+      const float m_new = fmaxf(m, tmax * scale_log2);   // scale_log2 > 0
       const bool raise = m_new > m + RESCALE_THRESHOLD;
       float alpha = 1.f;
       if (raise) {
-        alpha = exp2f(m - m_new);   // 0 on the first tile (m = -inf)
+        alpha = ex2_approx(m - m_new);   // 0 on the first tile (m = -inf)
         m = m_new;
       }
       l *= alpha;
       uint32_t pk[64];
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const float p0 = exp2f(s[2 * e] - m), p1 = exp2f(s[2 * e + 1] - m);
-        ls0 += p0;
-        ls1 += p1;
-        pk[e] = pack_bf16x2(p0, p1);
-      }
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), scale_log2, -m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), scale_log2, -m));
+          ls0 += p0;
+          ls1 += p1;
+          pk[c * 16 + e] = pack_bf16x2(p0, p1);
+        }
       l += ls0 + ls1;
 
       if (j > 0) {   // PV of the previous tile done: O is stable and the P buffer is free

@@ -253,7 +253,42 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr) {
 }
 
 // ------------------------------------------------------------------ math
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// 2^x with the SFU's approximate exponential (relative error about 2^-22,
+// results below 2^-126 flushed to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// erf(x) by the rational-exponential approximation 7.1.26 of Abramowitz and
+// Stegun, Handbook of Mathematical Functions (1964): for x >= 0,
+//   erf(x) ~= 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),
+//   t = 1 / (1 + p x),
+// with |error| <= 1.5e-7 over all x; odd symmetry for x < 0. Branch-free,
+// one reciprocal and one exponential on the SFU.
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  const float t = rcp_approx(fmaf(0.3275911f, ax, 1.0f));
+  float poly = fmaf(t, 1.061405429f, -1.453152027f);
+  poly = fmaf(t, poly, 1.421413741f);
+  poly = fmaf(t, poly, -0.284496736f);
+  poly = fmaf(t, poly, 0.254829592f);
+  poly *= t;
+  const float e = ex2_approx(-ax * ax * 1.4426950408889634f);
+  return copysignf(fmaf(-poly, e, 1.0f), x);
+}
+
+// Exact-form GELU, x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), with erf
+// evaluated by erf_as7126 (absolute error a few 1e-7, far below the bf16
+// rounding of the activations it produces).
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erf_as7126(x * 0.70710678118654752f)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -238,8 +238,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int row = row0 + lane;
       const bool row_ok = row < M;
       const int cbase = n0 + half * L::COLS_PER_WARP;
-
-      float run_max = -INFINITY, run_sum = 0.f, tgt_val = 0.f;
+      const int nvalid = min(L::COLS_PER_WARP, N - cbase);   // may be <= 0 (warp-uniform)
       int tgt = -1;
       if (EPI == EPI_LMHEAD) tgt = (row_ok && args.targets != nullptr) ? args.targets[row] : -1;
 
@@ -252,121 +251,149 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * L::COLS_PER_WARP;
-
-#pragma unroll 1
-      for (int c = 0; c < L::CHUNKS; ++c) {
-        const int col0 = cbase + c * 32;
-        if (col0 >= N) break;   // warp-uniform
-        float bias[32];
-        if (EPI != EPI_LMHEAD) load_bias32(static_cast<const bf16*>(args.bias), col0, N, bias);
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
+      // lm_head: pull this warp's whole slice of the accumulator into registers
+      // with a single wait and give the TMEM buffer back before any arithmetic.
+      uint32_t r[EPI == EPI_LMHEAD ? L::CHUNKS : 1][32];
+      if (EPI == EPI_LMHEAD) {
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c)
+          if (c * 32 < nvalid) tmem_ld_32x32b_x32(t_row + c * 32, r[c]);
         tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      }
 
-        if (EPI == EPI_BIAS || EPI == EPI_GELU) {
-          uint32_t pk[16];
+      if (EPI == EPI_LMHEAD) {
+        // log-sum-exp partial of this row over the valid columns of the half tile
+        float mx = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float a = v[2 * j] + bias[2 * j], b = v[2 * j + 1] + bias[2 * j + 1];
-            if (EPI == EPI_GELU) {
-              a = gelu_erf(a);
-              b = gelu_erf(b);
-            }
-            pk[j] = pack_bf16x2(a, b);
-          }
-          if (store_pending) {       // the previous chunk's TMA store must have read the buffer
-            if (lane == 0) bulk_wait_read_all();
-            __syncwarp();
-          }
-          // 32 rows x 64 B, 64-byte swizzle: 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_shared_v4(sb + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
-                         pk[4 * j + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row0 < M) {
-            tma_store_2d(&tmC, sbuf, col0, row0);
-            bulk_commit();
-          }
-          store_pending = true;
-        } else if (EPI == EPI_RESID) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] += bias[j];
-          if (store_pending) {
-            if (lane == 0) bulk_wait_read_all();
-            __syncwarp();
-          }
-          // 32 rows x 128 B, 128-byte swizzle: unit j of row r at unit j ^ (r & 7)
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_v4(sb + lane * 128 + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]),
-                         __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row0 < M) {
-            tma_reduce_add_2d(&tmC, sbuf, col0, row0);
-            bulk_commit();
-          }
-          store_pending = true;
-        } else {  // EPI_LMHEAD
-          const int nvalid = min(32, N - col0);
-          float cmax = -INFINITY;
+        for (int c = 0; c < L::CHUNKS; ++c)
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < nvalid) cmax = fmaxf(cmax, v[j]);
-          const float new_max = fmaxf(run_max, cmax);
-          const float nm2 = new_max * LOG2E;
-          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            if (c * 32 + j < nvalid) mx = fmaxf(mx, __uint_as_float(r[c][j]));
+        const float nm2 = mx * LOG2E;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c)
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
-            if (j + 0 < nvalid) s0 += exp2f(fmaf(v[j + 0], LOG2E, -nm2));
-            if (j + 1 < nvalid) s1 += exp2f(fmaf(v[j + 1], LOG2E, -nm2));
-            if (j + 2 < nvalid) s2 += exp2f(fmaf(v[j + 2], LOG2E, -nm2));
-            if (j + 3 < nvalid) s3 += exp2f(fmaf(v[j + 3], LOG2E, -nm2));
+            if (c * 32 + j + 0 < nvalid) s0 += ex2_approx(fmaf(__uint_as_float(r[c][j + 0]), LOG2E, -nm2));
+            if (c * 32 + j + 1 < nvalid) s1 += ex2_approx(fmaf(__uint_as_float(r[c][j + 1]), LOG2E, -nm2));
+            if (c * 32 + j + 2 < nvalid) s2 += ex2_approx(fmaf(__uint_as_float(r[c][j + 2]), LOG2E, -nm2));
+            if (c * 32 + j + 3 < nvalid) s3 += ex2_approx(fmaf(__uint_as_float(r[c][j + 3]), LOG2E, -nm2));
           }
-          run_sum = run_sum * exp2f(run_max * LOG2E - nm2) + ((s0 + s1) + (s2 + s3));
-          run_max = new_max;
-          const int tj = tgt - col0;
-          if (tj >= 0 && tj < 32) {
+        const int tj = tgt - cbase;
+        float tgt_val = 0.f;
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          const bool mine = tj >= c * 32 && tj < c * 32 + 32;
+          if (__any_sync(0xffffffffu, mine)) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j == tj) tgt_val = v[j];
+              if (mine && tj == c * 32 + j) tgt_val = __uint_as_float(r[c][j]);
           }
-          if (args.out != nullptr) {
-            // Transpose through shared memory (128-byte swizzled rows) so that
-            // each logits row segment is written by 32 consecutive lanes: the
-            // logits row pitch V is odd, so rows are only 4-byte aligned.
+        }
+        if (nvalid > 0 && row_ok) {
+          // one partial per (row, half tile): rows of `part` are column groups of BN/2
+          args.part[(size_t)(n_blk * 2 + half) * M + row] = make_float2(mx, (s0 + s1) + (s2 + s3));
+          if (tj >= 0 && tj < nvalid) args.tgt_logit[row] = tgt_val;
+        } else if (row_ok) {
+          args.part[(size_t)(n_blk * 2 + half) * M + row] = make_float2(-INFINITY, 0.f);
+        }
+        if (args.out != nullptr) {
+          // fp32 logits. The row pitch V is odd, so rows are only 4-byte
+          // aligned and neither vector nor TMA stores apply; short unaligned
+          // row pieces leave partial 32-byte sectors that write slowly. So
+          // each row's 128 columns leave as one contiguous 512-byte run:
+          // 8 rows at a time are transposed through this warp's 4 KB of
+          // shared memory (row rr at rr * 512, 16-byte unit u stored at
+          // unit u ^ rr, conflict-free both ways) and written by all 32 lanes
+          // as four back-to-back 128-byte stores per row.
+          float* lg = static_cast<float*>(args.out);
+#pragma unroll 1
+          for (int g = 0; g < 4; ++g) {
+            if ((lane >> 3) == g) {
+              const int rr = lane & 7;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              st_shared_v4(sb + lane * 128 + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]),
-                           __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
-                           __float_as_uint(v[4 * j + 3]));
+              for (int u = 0; u < 8 * L::CHUNKS; ++u)
+                st_shared_v4(sb + rr * 512 + ((u ^ rr) << 4), r[u >> 3][4 * (u & 7)], r[u >> 3][4 * (u & 7) + 1],
+                             r[u >> 3][4 * (u & 7) + 2], r[u >> 3][4 * (u & 7) + 3]);
+            }
             __syncwarp();
-            float* lg = static_cast<float*>(args.out);
-            const int gcol = col0 + lane;
-            const bool col_ok = gcol < N;
-#pragma unroll 8
-            for (int rr = 0; rr < 32; ++rr) {
-              const float val = ld_shared_f32(sb + rr * 128 + (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
-              if (row0 + rr < M && col_ok) lg[(size_t)(row0 + rr) * args.ldo + gcol] = val;
+#pragma unroll 2
+            for (int rr = 0; rr < 8; ++rr) {
+              const int grow = row0 + g * 8 + rr;
+              float* dst = lg + (size_t)grow * args.ldo + cbase;
+#pragma unroll
+              for (int k = 0; k < L::CHUNKS; ++k) {
+                const int e = 32 * k + lane;
+                const float val = ld_shared_f32(sb + rr * 512 + (((8 * k + (lane >> 2)) ^ rr) << 4) + ((lane & 3) << 2));
+                if (grow < M && e < nvalid) dst[e] = val;
+              }
             }
             __syncwarp();
           }
         }
-      }
-      // Accumulator fully read: hand it back to the MMA warp.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-
-      if (EPI == EPI_LMHEAD && row_ok) {
-        // one partial per (row, half tile): rows of `part` are column groups of BN/2
-        args.part[(size_t)(n_blk * 2 + half) * M + row] = make_float2(run_max, run_sum);
-        if (tgt >= cbase && tgt < cbase + L::COLS_PER_WARP && tgt < N) args.tgt_logit[row] = tgt_val;
+      } else {
+        // bias / GELU / residual: one 32-column chunk at a time (TMEM load,
+        // bias, activation, swizzled staging, TMA store or reduce-add)
+#pragma unroll 1
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          if (c * 32 >= nvalid) break;   // warp-uniform
+          const int col0 = cbase + c * 32;
+          float bias[32];
+          load_bias32(static_cast<const bf16*>(args.bias), col0, N, bias);
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_row + c * 32, v);
+          tmem_ld_wait();
+          uint32_t pk[32];
+          if (EPI == EPI_RESID) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pk[j] = __float_as_uint(__uint_as_float(v[j]) + bias[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float a = __uint_as_float(v[2 * j]) + bias[2 * j], b = __uint_as_float(v[2 * j + 1]) + bias[2 * j + 1];
+              if (EPI == EPI_GELU) {
+                a = gelu_erf(a);
+                b = gelu_erf(b);
+              }
+              pk[j] = pack_bf16x2(a, b);
+            }
+          }
+          if (store_pending) {       // the previous TMA store must have read the staging buffer
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
+          if (EPI == EPI_RESID) {
+            // 32 rows x 128 B, 128-byte swizzle: unit j of row r at unit j ^ (r & 7)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(sb + lane * 128 + ((j ^ (lane & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                           pk[4 * j + 3]);
+          } else {
+            // 32 rows x 64 B, 64-byte swizzle: unit j of row r at unit j ^ ((r >> 1) & 3)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(sb + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                           pk[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M) {
+            if (EPI == EPI_RESID)
+              tma_reduce_add_2d(&tmC, sbuf, col0, row0);
+            else
+              tma_store_2d(&tmC, sbuf, col0, row0);
+            bulk_commit();
+          }
+          store_pending = true;
+        }
+        // Accumulator fully read: hand it back to the MMA warp.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
       }
     }
     if (EPI != EPI_LMHEAD && lane == 0) bulk_wait_all();
