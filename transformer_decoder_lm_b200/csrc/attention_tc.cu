@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_wait();   // qkv comes from the previous kernel
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -213,11 +214,14 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
           for (int e = 0; e < 32; ++e)
             if (key0 + c * 32 + e > i || key0 + c * 32 + e >= T) sr[c][e] = __float_as_uint(-INFINITY);
       }
-      float tmax = -INFINITY;
+      float pm[8];   // 8 independent partial maxima keep the dependency chains short
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pm[e] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(sr[c][e]));
+        for (int e = 0; e < 32; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(sr[c][e]));
+      const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       const float m_new = fmaxf(m, tmax * scale_log2);   // scale_log2 > 0
       const bool raise = m_new > m + RESCALE_THRESHOLD;
       float alpha = 1.f;
@@ -227,18 +231,18 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
       }
       l *= alpha;
       uint32_t pk[64];
-      float ls0 = 0.f, ls1 = 0.f;
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), scale_log2, -m));
           const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), scale_log2, -m));
-          ls0 += p0;
-          ls1 += p1;
+          ls[(2 * e) & 7] += p0;
+          ls[(2 * e + 1) & 7] += p1;
           pk[c * 16 + e] = pack_bf16x2(p0, p1);
         }
-      l += ls0 + ls1;
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
 
       if (j > 0) {   // PV of the previous tile done: O is stable and the P buffer is free
         if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag)) {
@@ -304,6 +308,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0) pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
@@ -328,8 +333,8 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
     return cudaErrorInvalidValue;
   const int QT = (T + AT_BQ - 1) / AT_BQ;
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)AT_D));
-  attn_fwd_tc_kernel<<<B * H * QT, AT_THREADS, AT_SMEM, s>>>(tq, ty, B, T, H, C, scale_log2, status);
-  return cudaGetLastError();
+  return launch_pdl(attn_fwd_tc_kernel, dim3(B * H * QT), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
+                    status);
 }
 
 }  // namespace g2

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) ce_rows_kernel(const float2* __restrict__
                                                       float* __restrict__ token_loss, int* status) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   if (row >= M) return;
   float m = -INFINITY, s = 0.f;
   for (int i = lane; i < n_tiles; i += 32) {
@@ -56,6 +58,8 @@ __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__
                                                        float* __restrict__ loss_out, int* status) {
   __shared__ double ssum[32];
   __shared__ int scnt[32];
+  pdl_wait();
+  pdl_trigger();
   double acc = 0.0;
   int cnt = 0;
   for (int r = threadIdx.x; r < M; r += blockDim.x) {
@@ -99,9 +103,11 @@ __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__
 cudaError_t ce_finish_launch(const float2* part, int n_tiles, const float* tgt_logit, const int* targets, int M,
                              int V, float* token_loss, float* loss_out, int* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  ce_rows_kernel<<<(M + 7) / 8, 256, 0, s>>>(part, n_tiles, tgt_logit, targets, M, V, token_loss, status);
-  if (loss_out) ce_mean_kernel<<<1, 1024, 0, s>>>(token_loss, targets, M, V, loss_out, status);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(ce_rows_kernel, dim3((M + 7) / 8), dim3(256), 0, s, part, n_tiles, tgt_logit, targets, M,
+                             V, token_loss, status);
+  if (e == cudaSuccess && loss_out)
+    e = launch_pdl(ce_mean_kernel, dim3(1), dim3(1024), 0, s, token_loss, targets, M, V, loss_out, status);
+  return e;
 }
 
 }  // namespace g2

@@ -41,6 +41,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels of the forward pass are launched with programmatic stream
+// serialisation: a kernel may start (set up barriers, allocate TMEM, prefetch
+// descriptors) while its predecessor drains, and waits in pdl_wait() until
+// the predecessor has completed and its writes are visible before it reads
+// any of them. Each CTA calls pdl_trigger() once its last output is issued so
+// that the successor can be scheduled. Both are no-ops for plain launches.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -267,28 +277,30 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// erf(x) by the rational-exponential approximation 7.1.26 of Abramowitz and
-// Stegun, Handbook of Mathematical Functions (1964): for x >= 0,
-//   erf(x) ~= 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),
-//   t = 1 / (1 + p x),
-// with |error| <= 1.5e-7 over all x; odd symmetry for x < 0. Branch-free,
-// one reciprocal and one exponential on the SFU.
-__device__ __forceinline__ float erf_as7126(float x) {
-  const float ax = fabsf(x);
-  const float t = rcp_approx(fmaf(0.3275911f, ax, 1.0f));
-  float poly = fmaf(t, 1.061405429f, -1.453152027f);
-  poly = fmaf(t, poly, 1.421413741f);
-  poly = fmaf(t, poly, -0.284496736f);
-  poly = fmaf(t, poly, 0.254829592f);
-  poly *= t;
-  const float e = ex2_approx(-ax * ax * 1.4426950408889634f);
-  return copysignf(fmaf(-poly, e, 1.0f), x);
-}
-
 // Exact-form GELU, x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), with erf
-// evaluated by erf_as7126 (absolute error a few 1e-7, far below the bf16
-// rounding of the activations it produces).
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erf_as7126(x * 0.70710678118654752f)); }
+// evaluated by approximation 7.1.28 of Abramowitz and Stegun, Handbook of
+// Mathematical Functions (1964): for z >= 0,
+//   erf(z) ~= 1 - 1 / (1 + a1 z + a2 z^2 + a3 z^3 + a4 z^4 + a5 z^5 + a6 z^6)^16,
+// |error| <= 3e-7 (far below the bf16 rounding of the activations it feeds).
+// With r = 1 / (...)^16 ~= erfc(|z|), 1 + erf(z) is 2 - r for z >= 0 and r
+// for z < 0 (no cancellation for negative inputs). Branch-free, one SFU
+// reciprocal; a huge |z| makes the power overflow to inf and r = 0.
+__device__ __forceinline__ float gelu_erf(float x) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  float p = fmaf(z, 4.30638e-5f, 2.765672e-4f);
+  p = fmaf(z, p, 1.520143e-4f);
+  p = fmaf(z, p, 9.2705272e-3f);
+  p = fmaf(z, p, 4.22820123e-2f);
+  p = fmaf(z, p, 7.05230784e-2f);
+  p = fmaf(z, p, 1.0f);
+  p = p * p;   // ^2
+  p = p * p;   // ^4
+  p = p * p;   // ^8
+  p = p * p;   // ^16
+  const float r = rcp_approx(p);
+  const float one_plus_erf = x >= 0.f ? 2.0f - r : r;
+  return 0.5f * x * one_plus_erf;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -46,7 +46,11 @@ __global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids,
   const int warps = blockDim.x >> 5;
   const int row = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= M) return;
+  pdl_wait();
+  if (row >= M) {
+    pdl_trigger();
+    return;
+  }
   int id = ids[row];
   if (id < 0 || id >= V) {
     if (lane == 0) record_error(status, DEV_BAD_TOKEN);
@@ -61,6 +65,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids,
     const float4 b = Vec4<T>::load(pe + c);
     Vec4<float>::store(xr + c, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
   }
+  pdl_trigger();
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -77,7 +82,11 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
   const int warps = blockDim.x >> 5;
   const int row = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= M) return;
+  pdl_wait();
+  if (row >= M) {
+    pdl_trigger();
+    return;
+  }
   const float* xr = x + (size_t)row * C;
   float4 v[MAXV];
   float s = 0.f;
@@ -116,6 +125,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
       Vec4<T>::store(orow + c, o);
     }
   }
+  pdl_trigger();
 }
 
 cudaError_t embed_launch(bool bf16_, const int* ids, const void* wte, const void* wpe, float* x, int M, int T,
@@ -124,8 +134,8 @@ cudaError_t embed_launch(bool bf16_, const int* ids, const void* wte, const void
   const int threads = 256, rows_per_block = threads / 32;
   const int grid = (M + rows_per_block - 1) / rows_per_block;
   if (bf16_)
-    embed_kernel<bf16><<<grid, threads, 0, s>>>(ids, static_cast<const bf16*>(wte), static_cast<const bf16*>(wpe),
-                                                 x, M, T, C, V, status);
+    return launch_pdl(embed_kernel<bf16>, grid, threads, 0, s, ids, static_cast<const bf16*>(wte),
+                      static_cast<const bf16*>(wpe), x, M, T, C, V, status);
   else
     embed_kernel<float><<<grid, threads, 0, s>>>(ids, static_cast<const float*>(wte),
                                                   static_cast<const float*>(wpe), x, M, T, C, V, status);
@@ -140,11 +150,10 @@ cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const vo
   const int grid = (M + rows_per_block - 1) / rows_per_block;
   if (bf16_) {
     if (C <= 1024)
-      layernorm_kernel<bf16, 8><<<grid, threads, 0, s>>>(x, static_cast<const bf16*>(g), static_cast<const bf16*>(b),
-                                                         static_cast<bf16*>(out), M, C);
-    else
-      layernorm_kernel<bf16, 16><<<grid, threads, 0, s>>>(x, static_cast<const bf16*>(g),
-                                                          static_cast<const bf16*>(b), static_cast<bf16*>(out), M, C);
+      return launch_pdl(layernorm_kernel<bf16, 8>, grid, threads, 0, s, x, static_cast<const bf16*>(g),
+                        static_cast<const bf16*>(b), static_cast<bf16*>(out), M, C);
+    return launch_pdl(layernorm_kernel<bf16, 16>, grid, threads, 0, s, x, static_cast<const bf16*>(g),
+                      static_cast<const bf16*>(b), static_cast<bf16*>(out), M, C);
   } else {
     if (C <= 1024)
       layernorm_kernel<float, 8><<<grid, threads, 0, s>>>(x, static_cast<const float*>(g),

@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_wait();   // the operands and the residual stream come from the previous kernel
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -266,23 +267,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
       if (EPI == EPI_LMHEAD) {
         // log-sum-exp partial of this row over the valid columns of the half tile
-        float mx = -INFINITY;
+        // 8 independent partial maxima / sums keep the dependency chains short;
+        // columns at or past N count as -inf (exp2 gives 0)
+        float pm[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pm[j] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < L::CHUNKS; ++c)
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j < nvalid) mx = fmaxf(mx, __uint_as_float(r[c][j]));
-        const float nm2 = mx * LOG2E;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-        for (int c = 0; c < L::CHUNKS; ++c)
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            if (c * 32 + j + 0 < nvalid) s0 += ex2_approx(fmaf(__uint_as_float(r[c][j + 0]), LOG2E, -nm2));
-            if (c * 32 + j + 1 < nvalid) s1 += ex2_approx(fmaf(__uint_as_float(r[c][j + 1]), LOG2E, -nm2));
-            if (c * 32 + j + 2 < nvalid) s2 += ex2_approx(fmaf(__uint_as_float(r[c][j + 2]), LOG2E, -nm2));
-            if (c * 32 + j + 3 < nvalid) s3 += ex2_approx(fmaf(__uint_as_float(r[c][j + 3]), LOG2E, -nm2));
+          for (int j = 0; j < 32; ++j) {
+            if (c * 32 + j >= nvalid) r[c][j] = __float_as_uint(-INFINITY);
+            pm[j & 7] = fmaxf(pm[j & 7], __uint_as_float(r[c][j]));
           }
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float nm2 = mx * LOG2E;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ps[j & 7] += ex2_approx(fmaf(__uint_as_float(r[c][j]), LOG2E, -nm2));
+        const float s0 = ps[0] + ps[1], s1 = ps[2] + ps[3], s2 = ps[4] + ps[5], s3 = ps[6] + ps[7];
         const int tj = tgt - cbase;
         float tgt_val = 0.f;
 #pragma unroll
@@ -401,6 +405,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0) pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::TMEM_COLS);
@@ -443,8 +448,7 @@ cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUten
   const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
   const int grid = std::min(tiles, num_sms);
   if (grid <= 0) return cudaSuccess;
-  gemm_tc_kernel<BN, EPI><<<grid, TC_THREADS, L::SMEM_BYTES, s>>>(tA, tB, tC, a);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(TC_THREADS), L::SMEM_BYTES, s, tA, tB, tC, a);
 }
 
 template <int BN, int EPI>
