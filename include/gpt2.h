@@ -57,7 +57,8 @@ enum {
   GPT2_ERR_WORKSPACE = 4,       /* workspace too small or misaligned (256 B) */
   GPT2_ERR_BAD_TOKEN = 5,       /* device: an id was outside [0, vocab); it was clamped to 0 */
   GPT2_ERR_DEVICE_TIMEOUT = 6,  /* device: a bounded wait inside a kernel gave up */
-  GPT2_ERR_NO_TARGETS = 7       /* device: no position had a target >= 0; the loss was written as NaN */
+  GPT2_ERR_NO_TARGETS = 7,      /* device: no position had a target >= 0; the loss was written as NaN */
+  GPT2_ERR_SCRATCH_LIMIT = 8    /* the request needs more scratch than the allocation-free entry point holds */
 };
 
 /* Model shape. n_ctx is the size of the learned position table wpe
@@ -202,6 +203,29 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
                       int M, int C, int V, float* logits_or_null, float* token_loss_or_null,
                       float* loss_out, void* workspace, size_t ws_bytes, int* status,
                       void* stream);
+
+/* Allocation-free variant of gpt2_op_lmhead_ce. There is no counterpart in
+ * the pages: this exists for callers that cannot call cudaMalloc, such as a
+ * plugin inside a host application that owns every device allocation, or a
+ * latency-critical path on which cudaMalloc's implicit device
+ * synchronisation is not acceptable. Same arguments and results as
+ * gpt2_op_lmhead_ce, minus the workspace: the scratch is a fixed device
+ * array of GPT2_NOALLOC_SCRATCH_BYTES inside this library, held on every GPU
+ * that loads the library until the process exits. A call needs
+ * gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V) of it (about
+ * 16 * ceil(V / 128) bytes per row; V = 50257 allows up to 5335 rows); larger
+ * requests return GPT2_ERR_SCRATCH_LIMIT before any launch. The first call
+ * on each device performs a one-time set-up there (it looks up the array's
+ * device address, reads the SM count and sets kernel attributes), so make
+ * that first call before any stream capture. All calls share the one array
+ * and it keeps the last call's contents (no part of it needs to start at
+ * zero): calls whose kernels overlap on the GPU race on it, so order them on
+ * one stream. Never allocates device memory. */
+#define GPT2_NOALLOC_SCRATCH_BYTES (32u << 20)
+int gpt2_op_lmhead_ce_noalloc(int dtype, const void* hf, const void* wte, const int32_t* targets,
+                              int M, int C, int V, float* logits_or_null,
+                              float* token_loss_or_null, float* loss_out, int* status,
+                              void* stream);
 
 #ifdef __cplusplus
 }

@@ -12,5 +12,6 @@ from .binding import (  # noqa: F401
     gpt2_error_string, gpt2_destroy, gpt2_launch_count, gpt2_set_timing_events, GPT2_TIMED_LMHEAD,
     gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear,
     gpt2_op_attention, gpt2_op_lmhead_ce_workspace_bytes, gpt2_op_lmhead_ce, make_config,
+    gpt2_op_lmhead_ce_noalloc, GPT2_NOALLOC_SCRATCH_BYTES,
 )
 from .model import GPT2Model, upload_weights  # noqa: F401

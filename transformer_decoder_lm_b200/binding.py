@@ -21,7 +21,9 @@ GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID = 0, 1, 2
 ERRORS = {
     0: "GPT2_OK", 1: "GPT2_ERR_INVALID_ARG", 2: "GPT2_ERR_UNSUPPORTED", 3: "GPT2_ERR_CUDA",
     4: "GPT2_ERR_WORKSPACE", 5: "GPT2_ERR_BAD_TOKEN", 6: "GPT2_ERR_DEVICE_TIMEOUT", 7: "GPT2_ERR_NO_TARGETS",
+    8: "GPT2_ERR_SCRATCH_LIMIT",
 }
+GPT2_NOALLOC_SCRATCH_BYTES = 32 << 20
 ERR_CODE = {v: k for k, v in ERRORS.items()}
 
 LAYER_KEYS = (
@@ -74,6 +76,7 @@ def _load():
         "gpt2_op_attention": (i, [i, vp, i, i, i, i, vp, vp, vp]),
         "gpt2_op_lmhead_ce_workspace_bytes": (sz, [i, i, i]),
         "gpt2_op_lmhead_ce": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
+        "gpt2_op_lmhead_ce_noalloc": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -205,3 +208,13 @@ def gpt2_op_lmhead_ce(dtype, hf, wte, targets, M, C, V, logits, token_loss, loss
     _check(lib.gpt2_op_lmhead_ce(dtype, _ptr(hf), _ptr(wte), _ptr(targets), M, C, V, _ptr(logits), _ptr(token_loss),
                                  _ptr(loss_out), _ptr(workspace), nbytes, _ptr(status), _stream(stream)),
            "gpt2_op_lmhead_ce")
+
+
+def gpt2_op_lmhead_ce_noalloc(dtype, hf, wte, targets, M, C, V, logits, token_loss, loss_out, status=None,
+                              stream=None):
+    """gpt2_op_lmhead_ce without a workspace: for callers that cannot allocate
+    device memory; its scratch is a fixed array inside libgpt2.so (see
+    include/gpt2.h for the size limit and the ordering rule)."""
+    _check(lib.gpt2_op_lmhead_ce_noalloc(dtype, _ptr(hf), _ptr(wte), _ptr(targets), M, C, V, _ptr(logits),
+                                         _ptr(token_loss), _ptr(loss_out), _ptr(status), _stream(stream)),
+           "gpt2_op_lmhead_ce_noalloc")

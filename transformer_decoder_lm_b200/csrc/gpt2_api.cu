@@ -386,6 +386,7 @@ const char* gpt2_error_string(int code) {
     case GPT2_ERR_BAD_TOKEN: return "token id or target outside [0, vocab)";
     case GPT2_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
     case GPT2_ERR_NO_TARGETS: return "no position had a target";
+    case GPT2_ERR_SCRATCH_LIMIT: return "request needs more than the fixed scratch of the allocation-free entry point";
   }
   return "unknown error";
 }
