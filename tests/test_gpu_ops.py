@@ -95,7 +95,7 @@ LINEAR_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("bn", ["64", "128", "256", ""])
+@pytest.mark.parametrize("bn", ["64", "128", "192", "256", ""])
 @pytest.mark.parametrize("epi", [0, 1, 2])
 @pytest.mark.parametrize("shape", LINEAR_SHAPES)
 def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
@@ -194,7 +194,7 @@ def test_attention(G, dtype, B, T, H, C):
 # ------------------------------------------------------- lm_head + cross-entropy
 
 
-@pytest.mark.parametrize("bn", ["64", "128", "256", ""])
+@pytest.mark.parametrize("bn", ["64", "128", "192", "256", ""])
 @pytest.mark.parametrize("M,C,V", [(300, 768, 1000), (128, 128, 50257)])
 def test_lmhead_ce_bf16(G, M, C, V, bn, monkeypatch):
     if bn:

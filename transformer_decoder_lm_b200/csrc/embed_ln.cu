@@ -20,17 +20,22 @@ template <typename T>
 struct Vec4;
 template <>
 struct Vec4<float> {
+  typedef float4 raw_t;   // four elements as stored
+  static __device__ __forceinline__ raw_t load_raw(const float* p) { return *reinterpret_cast<const float4*>(p); }
+  static __device__ __forceinline__ float4 to_f4(raw_t r) { return r; }
   static __device__ __forceinline__ float4 load(const float* p) { return *reinterpret_cast<const float4*>(p); }
   static __device__ __forceinline__ void store(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 };
 template <>
 struct Vec4<bf16> {
-  static __device__ __forceinline__ float4 load(const bf16* p) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
+  typedef uint2 raw_t;
+  static __device__ __forceinline__ raw_t load_raw(const bf16* p) { return *reinterpret_cast<const uint2*>(p); }
+  static __device__ __forceinline__ float4 to_f4(raw_t u) {
     const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
     const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
     return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
   }
+  static __device__ __forceinline__ float4 load(const bf16* p) { return to_f4(load_raw(p)); }
   static __device__ __forceinline__ void store(bf16* p, float4 v) {
     uint2 u;
     u.x = pack_bf16x2(v.x, v.y);
@@ -76,7 +81,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // C <= 32 lanes * 4 * MAXV = 2048.
 template <typename T, int MAXV>
-__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, const T* __restrict__ g,
+__global__ void __launch_bounds__(128) layernorm_kernel(const float* __restrict__ x, const T* __restrict__ g,
                                                         const T* __restrict__ b, T* __restrict__ out, int M,
                                                         int C) {
   const int warps = blockDim.x >> 5;
@@ -88,15 +93,24 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
     return;
   }
   const float* xr = x + (size_t)row * C;
+  // x, gamma and beta are all requested before any of them is used, so a row
+  // costs one memory round trip.
   float4 v[MAXV];
-  float s = 0.f;
+  typename Vec4<T>::raw_t gg[MAXV], bt[MAXV];
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int c = (lane + 32 * i) * 4;
     if (c < C) {
       v[i] = Vec4<float>::load(xr + c);
-      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+      gg[i] = Vec4<T>::load_raw(g + c);
+      bt[i] = Vec4<T>::load_raw(b + c);
     }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
   }
   const float mean = warp_sum(s) / (float)C;
   float q = 0.f;
@@ -115,13 +129,12 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
   for (int i = 0; i < MAXV; ++i) {
     const int c = (lane + 32 * i) * 4;
     if (c < C) {
-      const float4 gg = Vec4<T>::load(g + c);
-      const float4 bt = Vec4<T>::load(b + c);
+      const float4 ga = Vec4<T>::to_f4(gg[i]), be = Vec4<T>::to_f4(bt[i]);
       float4 o;
-      o.x = (v[i].x - mean) * rstd * gg.x + bt.x;
-      o.y = (v[i].y - mean) * rstd * gg.y + bt.y;
-      o.z = (v[i].z - mean) * rstd * gg.z + bt.z;
-      o.w = (v[i].w - mean) * rstd * gg.w + bt.w;
+      o.x = (v[i].x - mean) * rstd * ga.x + be.x;
+      o.y = (v[i].y - mean) * rstd * ga.y + be.y;
+      o.z = (v[i].z - mean) * rstd * ga.z + be.z;
+      o.w = (v[i].w - mean) * rstd * ga.w + be.w;
       Vec4<T>::store(orow + c, o);
     }
   }
@@ -146,14 +159,17 @@ cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const vo
                              cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   if (C > 2048 || (C & 3)) return cudaErrorInvalidValue;
-  const int threads = 256, rows_per_block = threads / 32;
+  const int threads = 128, rows_per_block = threads / 32;
   const int grid = (M + rows_per_block - 1) / rows_per_block;
   if (bf16_) {
-    if (C <= 1024)
-      return launch_pdl(layernorm_kernel<bf16, 8>, grid, threads, 0, s, x, static_cast<const bf16*>(g),
-                        static_cast<const bf16*>(b), static_cast<bf16*>(out), M, C);
-    return launch_pdl(layernorm_kernel<bf16, 16>, grid, threads, 0, s, x, static_cast<const bf16*>(g),
-                      static_cast<const bf16*>(b), static_cast<bf16*>(out), M, C);
+    // registers per lane grow with C: pick the smallest row capacity that fits
+    const bf16 *gp = static_cast<const bf16*>(g), *bp = static_cast<const bf16*>(b);
+    bf16* op = static_cast<bf16*>(out);
+    if (C <= 768) return launch_pdl(layernorm_kernel<bf16, 6>, grid, threads, 0, s, x, gp, bp, op, M, C);
+    if (C <= 1024) return launch_pdl(layernorm_kernel<bf16, 8>, grid, threads, 0, s, x, gp, bp, op, M, C);
+    if (C <= 1280) return launch_pdl(layernorm_kernel<bf16, 10>, grid, threads, 0, s, x, gp, bp, op, M, C);
+    if (C <= 1664) return launch_pdl(layernorm_kernel<bf16, 13>, grid, threads, 0, s, x, gp, bp, op, M, C);
+    return launch_pdl(layernorm_kernel<bf16, 16>, grid, threads, 0, s, x, gp, bp, op, M, C);
   } else {
     if (C <= 1024)
       layernorm_kernel<float, 8><<<grid, threads, 0, s>>>(x, static_cast<const float*>(g),

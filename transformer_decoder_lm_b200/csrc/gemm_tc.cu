@@ -501,25 +501,27 @@ bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t 
 int gemm_tc_n_tiles(int N, int bn) { return 2 * ((N + bn - 1) / bn); }
 
 int gemm_tc_pick_bn(int M, int N, int num_sms) {
-  // G2_GEMM_BN=64|128|256 pins the tile width (tests use it to cover every
-  // instantiation); otherwise the width is chosen by the cost model below.
+  // G2_GEMM_BN=64|128|192|256 pins the tile width (tests use it to cover
+  // every instantiation); otherwise the width is chosen by the cost model below.
   if (const char* e = getenv("G2_GEMM_BN")) {
     const int v = atoi(e);
-    if (v == 64 || v == 128 || v == 256) return v;
+    if (v == 64 || v == 128 || v == 192 || v == 256) return v;
   }
   // Estimated cost = waves x per-tile cost. Narrower tiles re-read A from
   // shared memory more often per FLOP (the 128-row MMA at N=128 runs at
-  // about 60% of the N=256 rate), so their per-column cost is higher.
-  const int cand[3] = {256, 128, 64};
-  const double unit[3] = {256.0, 200.0, 150.0};
+  // about 60% of the N=256 rate), so their per-column cost is higher; N=192
+  // still keeps the MMA's shared-memory reads under the per-SM bandwidth.
+  // A narrower width must win by more than 2% to be taken.
+  const int cand[4] = {256, 192, 128, 64};
+  const double unit[4] = {256.0, 192.0, 200.0, 150.0};
   const int mt = (M + TC_BM - 1) / TC_BM;
   int best = 256;
   double best_cost = 1e30;
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const long tiles = (long)mt * ((N + cand[i] - 1) / cand[i]);
     const long waves = (tiles + num_sms - 1) / num_sms;
     const double cost = waves * unit[i];
-    if (cost < best_cost - 1e-9) {
+    if (cost < best_cost * 0.98) {
       best_cost = cost;
       best = cand[i];
     }
@@ -531,6 +533,7 @@ cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tA, const CUtenso
                            const GemmArgs& a, int num_sms, cudaStream_t s) {
   switch (bn) {
     case 256: return launch_bn<256>(epi, tA, tB, tC, a, num_sms, s);
+    case 192: return launch_bn<192>(epi, tA, tB, tC, a, num_sms, s);
     case 128: return launch_bn<128>(epi, tA, tB, tC, a, num_sms, s);
     case 64: return launch_bn<64>(epi, tA, tB, tC, a, num_sms, s);
   }
@@ -545,6 +548,7 @@ cudaError_t gemm_tc_set_attributes() {
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID>();       \
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD>();
   G2_ATTR(256)
+  G2_ATTR(192)
   G2_ATTR(128)
   G2_ATTR(64)
 #undef G2_ATTR

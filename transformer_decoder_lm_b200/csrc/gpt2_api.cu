@@ -30,8 +30,9 @@ using namespace g2;
 
 namespace {
 
-constexpr int BN_CHOICES[3] = {256, 128, 64};
-inline int bn_index(int bn) { return bn == 256 ? 0 : (bn == 128 ? 1 : 2); }
+constexpr int NUM_BN = 4;
+constexpr int BN_CHOICES[NUM_BN] = {256, 192, 128, 64};
+inline int bn_index(int bn) { return bn == 256 ? 0 : (bn == 192 ? 1 : (bn == 128 ? 2 : 3)); }
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -45,7 +46,7 @@ struct LayerPtrs {
 };
 
 struct WeightMaps {  // one tensor map per candidate tile width
-  CUtensorMap attn[3], proj[3], fc[3], mproj[3];
+  CUtensorMap attn[NUM_BN], proj[NUM_BN], fc[NUM_BN], mproj[NUM_BN];
 };
 
 struct Plan {
@@ -122,7 +123,7 @@ struct gpt2_model {
   const void *wte = nullptr, *wpe = nullptr, *lnf_g = nullptr, *lnf_b = nullptr;
   std::vector<LayerPtrs> layers;
   std::vector<WeightMaps> maps;
-  CUtensorMap wte_map[3];
+  CUtensorMap wte_map[NUM_BN];
   uint8_t* ws = nullptr;
   Plan plan;
   float* x = nullptr;
@@ -323,7 +324,7 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
     const int C = cfg->n_embd;
     m->maps.resize(L);
     bool ok = true;
-    for (int i = 0; i < 3 && ok; ++i) {
+    for (int i = 0; i < NUM_BN && ok; ++i) {
       const uint32_t bn = BN_CHOICES[i];
       ok = ok && make_tmap_bf16(&m->wte_map[i], m->wte, cfg->vocab, C, C, bn);
       for (int l = 0; l < L && ok; ++l) {
