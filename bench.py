@@ -194,16 +194,14 @@ def run_ours(args):
     M = WL.batch * WL.seq
     logits = torch.empty(WL.batch, WL.seq, WL.vocab, dtype=torch.float32, device="cuda")
     loss = torch.empty(1, dtype=torch.float32, device="cuda")
-    red = torch.zeros(2, dtype=torch.float32, device="cuda")
     n_valid = float((tg_np >= 0).sum())
+
+    from transformer_decoder_lm_b200 import dist as gdist
 
     def step(i_ids, i_tg):
         G.gpt2_forward_loss(model.handle, i_ids, i_tg, WL.batch, WL.seq, logits, loss, None, stream)
-        if world > 1:
-            red[0:1].copy_(loss * n_valid)
-            red[1] = n_valid
-            dist.all_reduce(red)
-            loss.copy_(red[0:1] / red[1])
+        if world > 1:   # the one exchange of the data-parallel forward: the loss mean
+            loss.copy_(gdist.global_mean_loss(loss, int(n_valid)))
 
     def barrier():
         if world > 1:
@@ -241,9 +239,7 @@ def run_ours(args):
     if rc != 0:
         raise RuntimeError(f"device status after timing: {G.gpt2_error_string(rc)}")
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = gdist.max_over_ranks(ms, "cuda")
     ms_step = ms / args.steps
     tokens_all = M * world
     value = tokens_all / (ms_step / 1000.0)
@@ -273,9 +269,7 @@ def run_ours(args):
     barrier()
     ems = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ems], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
+        ems = gdist.max_over_ranks(ems, "cuda")
     e2e_value = tokens_all / (ems / args.steps / 1000.0)
 
     hbm, tf_burst, tf_sust, peak_kind = peaks()
