@@ -55,6 +55,35 @@ def lmhead_flops(wl, M) -> float:
     return 2.0 * M * wl.vocab * wl.n_embd
 
 
+LMHEAD_SOURCES = ("transformer_decoder_lm_b200/csrc/gemm_tc.cu", "transformer_decoder_lm_b200/csrc/common.cuh",
+                  "transformer_decoder_lm_b200/csrc/kernels.h")
+LMHEAD_PROFILE = "profiles/lm_head_tcgen05_124M.md"
+
+
+def lmhead_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in LMHEAD_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()
+
+
+def lmhead_traffic():
+    """DRAM bytes (read + write) per lm_head launch from the committed ncu
+    summary, or None if the summary is missing or was taken on other kernel
+    sources than the ones built now."""
+    import re
+    p = os.path.join(ROOT, LMHEAD_PROFILE)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != lmhead_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -288,7 +317,7 @@ def run_ours(args):
         "peak_note": f"{peak_kind} bf16 {tf_burst} TF/s burst, {tf_sust} sustained",
         "roofline": {"kernel": "lm_head tcgen05 GEMM + fused log-sum-exp (gemm_tc_kernel EPI_LMHEAD)",
                      "bound": "tensor", "achieved": lm_tflops, "peak": tf_sust, "unit": "TFLOP/s",
-                     "frac": lm_tflops / tf_sust, "traffic": None,
+                     "frac": lm_tflops / tf_sust, "traffic": lmhead_traffic(),
                      "flops_per_launch": lmhead_flops(WL, M), "ms_per_launch": lm_ms,
                      "peak_kind": f"{peak_kind} sustained (kernel timed inside a long step)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h_ids.numel() * 4 + h_tg.numel() * 4),
