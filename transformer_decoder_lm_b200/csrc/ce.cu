@@ -6,42 +6,51 @@
 // mean reduction over the shifted targets).
 //
 // The lm_head epilogue left, per row and column group, (m_i, s_i) with
-// s_i = sum over the group of exp(z - m_i). Here one warp per row merges them:
-// M = max m_i, S = sum s_i exp(m_i - M), lse = M + log S. A single block then
-// forms the mean in double precision in a fixed order (deterministic).
+// s_i = sum over the group of exp(z - m_i). ce_rows_kernel merges them per
+// row: M = max m_i, S = sum s_i exp(m_i - M), lse = M + log S. A single block
+// then forms the mean in double precision in a fixed order (deterministic).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace g2 {
 
+// One block per 32 rows: lane = row, so every load of a partial is a
+// coalesced 256-byte read of one column group for 32 consecutive rows; the 8
+// warps take the column groups round-robin and their running (max, sum) pairs
+// are merged through shared memory.
 __global__ void __launch_bounds__(256) ce_rows_kernel(const float2* __restrict__ part, int n_tiles,
                                                       const float* __restrict__ tgt_logit,
                                                       const int* __restrict__ targets, int M, int V,
                                                       float* __restrict__ token_loss, int* status) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  __shared__ float sm_m[8][32], sm_s[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 32 + lane;
   pdl_wait();
   pdl_trigger();
-  if (row >= M) return;
   float m = -INFINITY, s = 0.f;
-  for (int i = lane; i < n_tiles; i += 32) {
-    const float2 p = part[(size_t)i * M + row];
-    if (p.x == -INFINITY) continue;   // a column group with no valid column
-    const float mn = fmaxf(m, p.x);
-    s = s * expf(m - mn) + p.y * expf(p.x - mn);
-    m = mn;
+  if (row < M) {
+    for (int i = warp; i < n_tiles; i += 8) {
+      const float2 p = part[(size_t)i * M + row];
+      if (p.x == -INFINITY) continue;   // a column group with no valid column
+      const float mn = fmaxf(m, p.x);
+      s = s * expf(m - mn) + p.y * expf(p.x - mn);
+      m = mn;
+    }
   }
+  sm_m[warp][lane] = m;
+  sm_s[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && row < M) {
+    m = -INFINITY;
+    s = 0.f;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
-    const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
-    const float mn = fmaxf(m, m2);
-    const float a = (m == -INFINITY) ? 0.f : expf(m - mn);
-    const float a2 = (m2 == -INFINITY) ? 0.f : expf(m2 - mn);
-    s = s * a + s2 * a2;
-    m = mn;
-  }
-  if (lane == 0) {
+    for (int w = 0; w < 8; ++w) {
+      const float m2 = sm_m[w][lane], s2 = sm_s[w][lane];
+      if (m2 == -INFINITY) continue;
+      const float mn = fmaxf(m, m2);
+      s = s * expf(m - mn) + s2 * expf(m2 - mn);
+      m = mn;
+    }
     const int tg = targets[row];
     float l = 0.f;
     if (tg >= V) {
@@ -103,8 +112,8 @@ __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__
 cudaError_t ce_finish_launch(const float2* part, int n_tiles, const float* tgt_logit, const int* targets, int M,
                              int V, float* token_loss, float* loss_out, int* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = launch_pdl(ce_rows_kernel, dim3((M + 7) / 8), dim3(256), 0, s, part, n_tiles, tgt_logit, targets, M,
-                             V, token_loss, status);
+  cudaError_t e = launch_pdl(ce_rows_kernel, dim3((M + 31) / 32), dim3(256), 0, s, part, n_tiles, tgt_logit, targets,
+                             M, V, token_loss, status);
   if (e == cudaSuccess && loss_out)
     e = launch_pdl(ce_mean_kernel, dim3(1), dim3(1024), 0, s, token_loss, targets, M, V, loss_out, status);
   return e;
