@@ -188,7 +188,10 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
 
 /* Causal multi-head self-attention. qkv [B*T, 3C] (`dtype`, columns q | k | v,
  * head h at columns h*D..h*D+D-1 of each) -> y [B*T, C] (`dtype`), heads
- * concatenated. D = C / H must be 32 or 64. */
+ * concatenated. D = C / H must be 32 or 64. The bf16, D = 64 kernel schedules
+ * its work through a pair of counters that the library keeps per device, so
+ * calls of this entry point on one device must not overlap on the GPU (the
+ * model's own forward passes use counters in their workspace instead). */
 int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, void* y,
                       int* status, void* stream);
 

@@ -181,6 +181,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem desc]^T: A (M x 16 bf16 per instruction) read
+// from tensor memory, lanes = rows, each 32-bit column holding two
+// consecutive K elements (the lower one in the low half).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread
 // has completed (its smem operands may be overwritten, its TMEM result read).
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -276,6 +288,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for x <= 127 (inputs below -126 give about 2^-126): x = n + f
+// with n the nearest integer (by the 1.5 * 2^23 rounding trick) and
+// f in [-0.5, 0.5]; 2^f by a degree-4 polynomial fitted here for relative
+// error (max 2.7e-6 on that interval); 2^n added to the exponent field.
+// Used for a share of the softmax exponentials so that they do not all queue
+// on the SFU.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float fr = x - (t - 12582912.0f);
+  float p = fmaf(9.570068679749966e-3f, fr, 5.5917806923389435e-2f);
+  p = fmaf(p, fr, 2.40247443318367e-1f);
+  p = fmaf(p, fr, 6.931218504905701e-1f);
+  p = fmaf(p, fr, 9.999992847442627e-1f);
+  // low bits of t hold n (two's complement); shifting them into the exponent
+  // field is done in unsigned arithmetic (wrap-around is intended)
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 __device__ __forceinline__ float rcp_approx(float x) {

@@ -132,6 +132,7 @@ struct gpt2_model {
   float* tgt = nullptr;
   float* tok = nullptr;
   int* status = nullptr;
+  unsigned* sched = nullptr;   // attention work counters (in the zeroed status block)
   uint64_t launches = 0;
   cudaEvent_t ev_lm_begin = nullptr, ev_lm_end = nullptr;
 };
@@ -196,7 +197,7 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
     G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C, m->qkv, 3 * C, s));
-    G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, m->status, s));
+    G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, m->sched, m->status, s));
     G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
     G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, &out_f, L.fc_b, M, 4 * C, C, m->f, 4 * C, s));
@@ -319,6 +320,7 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
   m->tgt = reinterpret_cast<float*>(ws + p.tgt);
   m->tok = reinterpret_cast<float*>(ws + p.tok);
   m->status = reinterpret_cast<int*>(ws + p.status);
+  m->sched = reinterpret_cast<unsigned*>(ws + p.status + 64);
 
   if (m->bf16) {
     const int C = cfg->n_embd;
@@ -464,7 +466,7 @@ int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, vo
     return GPT2_ERR_INVALID_ARG;
   const int D = C / H;
   if (D != 32 && D != 64) return GPT2_ERR_UNSUPPORTED;
-  return attention_launch(dtype == GPT2_BF16, qkv, y, B, T, H, C, status, static_cast<cudaStream_t>(stream)) ==
+  return attention_launch(dtype == GPT2_BF16, qkv, y, B, T, H, C, nullptr, status, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? GPT2_OK
              : GPT2_ERR_CUDA;

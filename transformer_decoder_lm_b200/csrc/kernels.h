@@ -80,9 +80,14 @@ cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const voi
 
 // ---- attention ---------------------------------------------------------------
 // tcgen05 flash attention (bf16, d_head 64); attention_launch dispatches to it.
-cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, int* status, cudaStream_t s);
-cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C, int* status,
-                             cudaStream_t s);
+// sched: two zeroed uint32 device counters the persistent kernel schedules its
+// work with (left zeroed again when it ends); NULL uses a per-device pair of
+// the library's own, shared by every launch that passes NULL (those launches
+// must not overlap).
+cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, unsigned* sched, int* status,
+                                cudaStream_t s);
+cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C, unsigned* sched,
+                             int* status, cudaStream_t s);
 
 // ---- cross-entropy finalisation -------------------------------------------
 // token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
