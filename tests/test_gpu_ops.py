@@ -175,8 +175,10 @@ def test_linear_fp32_simt(G, epi):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-@pytest.mark.parametrize("B,T,H,C", [(2, 200, 4, 256), (1, 64, 2, 64), (3, 1, 12, 768), (1, 333, 12, 768)])
+@pytest.mark.parametrize("B,T,H,C", [(2, 200, 4, 256), (1, 64, 2, 64), (3, 1, 12, 768), (1, 333, 12, 768),
+                                     (1, 1024, 12, 768), (2, 1000, 4, 256), (1, 2048, 2, 128)])
 def test_attention(G, dtype, B, T, H, C):
+    # the longer cases split their last query tiles into two key ranges merged at the end
     rng = np.random.default_rng(B * 1000 + T + H)
     qkv = bf16_exact(rng, (B * T, 3 * C))
     y = torch.empty(B * T, C, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device="cuda")
@@ -189,6 +191,10 @@ def test_attention(G, dtype, B, T, H, C):
     else:
         assert rel_l2(got, ref) <= 5e-3
         assert max_abs(got, ref) <= 2e-2
+        # a second launch (split flags and counters reset by the first) gives the same bits
+        y2 = torch.empty_like(y)
+        G.gpt2_op_attention(code, dev(qkv, dtype), B, T, H, C, y2)
+        assert torch.equal(y, y2)
 
 
 # ------------------------------------------------------- lm_head + cross-entropy

@@ -244,14 +244,14 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(const float* __restri
     if ((d & 31) == lane) yr[d] = o[d] * inv;
 }
 
-cudaError_t attention_launch(bool bf16_, const void* qkv, void* y, int B, int T, int H, int C, unsigned* sched,
-                             int* status, cudaStream_t s) {
+cudaError_t attention_launch(bool bf16_, const void* qkv, void* y, int B, int T, int H, int C,
+                             const AttnScratch* scratch, int* status, cudaStream_t s) {
   (void)status;
   if (B <= 0 || T <= 0) return cudaSuccess;
   const int D = C / H;
   if (bf16_) {
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    if (D == 64) return attention_tc_launch(qkv, y, B, T, H, C, sched, status, s);
+    if (D == 64) return attention_tc_launch(qkv, y, B, T, H, C, scratch, status, s);
     dim3 grid((T + 63) / 64, H, B);
     if (D == 64)
       attn_fwd_bf16_kernel<64><<<grid, 128, 0, s>>>(static_cast<const bf16*>(qkv), static_cast<bf16*>(y), T, H, C,

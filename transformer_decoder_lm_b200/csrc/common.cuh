@@ -309,6 +309,64 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
+// ---- packed fp32 pairs: on sm_100 one instruction adds, subtracts or
+// fuses-multiply-adds two floats held in a 64-bit register pair.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// ex2_poly on a pair of floats, the rounding split and the polynomial in
+// packed arithmetic (each lane the same IEEE operations as ex2_poly).
+__device__ __forceinline__ void ex2_poly_x2(uint64_t x, float& y0, float& y1) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(xc, magic);
+  const uint64_t fr = f2_sub(xc, f2_sub(t, magic));
+  uint64_t p = f2_fma(f2_pack(9.570068679749966e-3f, 9.570068679749966e-3f), fr,
+                      f2_pack(5.5917806923389435e-2f, 5.5917806923389435e-2f));
+  p = f2_fma(p, fr, f2_pack(2.40247443318367e-1f, 2.40247443318367e-1f));
+  p = f2_fma(p, fr, f2_pack(6.931218504905701e-1f, 6.931218504905701e-1f));
+  p = f2_fma(p, fr, f2_pack(9.999992847442627e-1f, 9.999992847442627e-1f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -338,6 +396,31 @@ __device__ __forceinline__ float gelu_erf(float x) {
   const float r = rcp_approx(p);
   const float one_plus_erf = x >= 0.f ? 2.0f - r : r;
   return 0.5f * x * one_plus_erf;
+}
+
+// gelu_erf on a pair in packed fp32. With r = 1 - erf(|x|/sqrt2) from the
+// same approximation, gelu(x) = 0.5 x (1 + erf(x/sqrt2)) = relu(x) - 0.5 |x| r
+// for either sign of x (x >= 0: x - 0.5 x r; x < 0: 0.5 x r).
+__device__ __forceinline__ uint64_t gelu_erf_x2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t z = f2_mul(f2_pack(fabsf(x0), fabsf(x1)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
+  uint64_t p = f2_fma(z, f2_pack(4.30638e-5f, 4.30638e-5f), f2_pack(2.765672e-4f, 2.765672e-4f));
+  p = f2_fma(z, p, f2_pack(1.520143e-4f, 1.520143e-4f));
+  p = f2_fma(z, p, f2_pack(9.2705272e-3f, 9.2705272e-3f));
+  p = f2_fma(z, p, f2_pack(4.22820123e-2f, 4.22820123e-2f));
+  p = f2_fma(z, p, f2_pack(7.05230784e-2f, 7.05230784e-2f));
+  p = f2_fma(z, p, f2_pack(1.0f, 1.0f));
+  p = f2_mul(p, p);   // ^2
+  p = f2_mul(p, p);   // ^4
+  p = f2_mul(p, p);   // ^8
+  p = f2_mul(p, p);   // ^16
+  float p0, p1;
+  f2_unpack(p, p0, p1);
+  const uint64_t r = f2_pack(rcp_approx(p0), rcp_approx(p1));
+  // -0.5 |x| = z * (-0.5 * sqrt2)
+  const uint64_t h = f2_mul(z, f2_pack(-0.70710678118654752f, -0.70710678118654752f));
+  return f2_fma(h, r, f2_pack(fmaxf(x0, 0.f), fmaxf(x1, 0.f)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // bias, activation, swizzled staging, TMA store or reduce-add)
 #pragma unroll 1
         for (int c = 0; c < L::CHUNKS; ++c) {
-          if (c * 32 >= nvalid) break;   // warp-uniform
+          if (c * 32 >= nvalid || row0 >= M) break;   // warp-uniform: nothing of this warp's rows to write
           const int col0 = cbase + c * 32;
           float bias[32];
           load_bias32(static_cast<const bf16*>(args.bias), col0, N, bias);
@@ -358,12 +358,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              float a = __uint_as_float(v[2 * j]) + bias[2 * j], b = __uint_as_float(v[2 * j + 1]) + bias[2 * j + 1];
               if (EPI == EPI_GELU) {
-                a = gelu_erf(a);
-                b = gelu_erf(b);
+                uint64_t y2 = f2_add(f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])),
+                                     f2_pack(bias[2 * j], bias[2 * j + 1]));
+                y2 = gelu_erf_x2(y2);
+                float a, b;
+                f2_unpack(y2, a, b);
+                pk[j] = pack_bf16x2(a, b);
+              } else {
+                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) + bias[2 * j], __uint_as_float(v[2 * j + 1]) + bias[2 * j + 1]);
               }
-              pk[j] = pack_bf16x2(a, b);
             }
           }
           if (store_pending) {       // the previous TMA store must have read the staging buffer
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && row0 < M) {
+          if (lane == 0) {
             if (EPI == EPI_RESID)
               tma_reduce_add_2d(&tmC, sbuf, col0, row0);
             else

@@ -50,10 +50,12 @@ struct WeightMaps {  // one tensor map per candidate tile width
 };
 
 struct Plan {
-  size_t x, h, qkv, y, f, part, tgt, tok, status, total;
+  size_t x, h, qkv, y, f, part, tgt, tok, attn, attn_flags, status, total;
+  int attn_pairs;
 };
 
-Plan plan_workspace(const gpt2_config_t& c, long M) {
+Plan plan_workspace(const gpt2_config_t& c, int max_B, int max_T) {
+  const long M = (long)max_B * max_T;
   const size_t es = c.dtype == GPT2_BF16 ? 2 : 4;
   const size_t C = (size_t)c.n_embd;
   const size_t n_tiles = lmhead_groups(c.vocab);
@@ -67,6 +69,12 @@ Plan plan_workspace(const gpt2_config_t& c, long M) {
   p.part = o;   o += align256(n_tiles * M * sizeof(float2));
   p.tgt = o;    o += align256(M * 4);
   p.tok = o;    o += align256(M * 4);
+  // attention split scratch: a flag block (zeroed at create) then the partials
+  p.attn_pairs = 0;
+  if (c.dtype == GPT2_BF16 && c.n_embd / c.n_head == 64)
+    p.attn_pairs = (int)(attention_scratch_bytes(max_B, max_T, c.n_head) / (ATTN_PART_FLOATS * 4 + ATTN_PAIR_FLAGS * 4));
+  p.attn_flags = o; o += align256((size_t)p.attn_pairs * ATTN_PAIR_FLAGS * 4);
+  p.attn = o;   o += align256((size_t)p.attn_pairs * ATTN_PART_FLOATS * 4);
   p.status = o; o += 256;
   p.total = o;
   return p;
@@ -132,7 +140,7 @@ struct gpt2_model {
   float* tgt = nullptr;
   float* tok = nullptr;
   int* status = nullptr;
-  unsigned* sched = nullptr;   // attention work counters (in the zeroed status block)
+  AttnScratch attn;            // attention work counters (in the zeroed status block), split flags, partials
   uint64_t launches = 0;
   cudaEvent_t ev_lm_begin = nullptr, ev_lm_end = nullptr;
 };
@@ -197,7 +205,7 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
     G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C, m->qkv, 3 * C, s));
-    G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, m->sched, m->status, s));
+    G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, &m->attn, m->status, s));
     G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
     G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, &out_f, L.fc_b, M, 4 * C, C, m->f, 4 * C, s));
@@ -250,7 +258,7 @@ extern "C" {
 
 size_t gpt2_workspace_bytes(const gpt2_config_t* cfg, int max_B, int max_T) {
   if (check_config(cfg) != GPT2_OK || max_B < 1 || max_T < 1) return 0;
-  return plan_workspace(*cfg, (long)max_B * max_T).total;
+  return plan_workspace(*cfg, max_B, max_T < cfg->n_ctx ? max_T : cfg->n_ctx).total;
 }
 
 int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspace, size_t ws_bytes, int max_B,
@@ -262,7 +270,7 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
   if (!w || !workspace || max_B < 1 || max_T < 1) return GPT2_ERR_INVALID_ARG;
   if (max_T > cfg->n_ctx) max_T = cfg->n_ctx;
   const long maxM = (long)max_B * max_T;
-  const Plan p = plan_workspace(*cfg, maxM);
+  const Plan p = plan_workspace(*cfg, max_B, max_T);
   if (ws_bytes < p.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return GPT2_ERR_WORKSPACE;
   const int L = cfg->n_layer;
   const void* const* arrays[12] = {w->ln1_g, w->ln1_b, w->attn_w,  w->attn_b, w->attn_proj_w, w->attn_proj_b,
@@ -320,7 +328,10 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
   m->tgt = reinterpret_cast<float*>(ws + p.tgt);
   m->tok = reinterpret_cast<float*>(ws + p.tok);
   m->status = reinterpret_cast<int*>(ws + p.status);
-  m->sched = reinterpret_cast<unsigned*>(ws + p.status + 64);
+  m->attn.sched = reinterpret_cast<unsigned*>(ws + p.status + 64);
+  m->attn.flags = reinterpret_cast<int*>(ws + p.attn_flags);
+  m->attn.part = reinterpret_cast<float*>(ws + p.attn);
+  m->attn.cap_pairs = p.attn_pairs;
 
   if (m->bf16) {
     const int C = cfg->n_embd;
@@ -341,7 +352,9 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
       return GPT2_ERR_CUDA;
     }
   }
-  if (cudaMemset(m->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+  if (cudaMemset(m->status, 0, 256) != cudaSuccess ||
+      (p.attn_pairs && cudaMemset(m->attn.flags, 0, (size_t)p.attn_pairs * ATTN_PAIR_FLAGS * 4) != cudaSuccess) ||
+      cudaDeviceSynchronize() != cudaSuccess) {
     delete m;
     return GPT2_ERR_CUDA;
   }

@@ -80,14 +80,31 @@ cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const voi
 
 // ---- attention ---------------------------------------------------------------
 // tcgen05 flash attention (bf16, d_head 64); attention_launch dispatches to it.
-// sched: two zeroed uint32 device counters the persistent kernel schedules its
-// work with (left zeroed again when it ends); NULL uses a per-device pair of
-// the library's own, shared by every launch that passes NULL (those launches
-// must not overlap).
-cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, unsigned* sched, int* status,
-                                cudaStream_t s);
-cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C, unsigned* sched,
-                             int* status, cudaStream_t s);
+// Scratch of the persistent kernel:
+//   sched      two zeroed uint32 counters it schedules its work with (left
+//              zeroed again when it ends);
+//   flags      cap_pairs * ATTN_PAIR_FLAGS zeroed int32 words (left zeroed again);
+//   part       cap_pairs * ATTN_PART_FLOATS floats, no initial contents.
+// The longest query tiles are split in two key ranges; the half that
+// finishes first leaves its unnormalised partial output in `part` for the
+// other to merge.
+// cap_pairs bounds how many (sequence, head, query tile) triples may split
+// (0: none). A NULL sched uses the library's own per-device scratch, shared by
+// every launch that passes NULL (those launches must not overlap).
+constexpr int ATTN_PART_FLOATS = 128 * 64 + 2 * 128;
+constexpr int ATTN_PAIR_FLAGS = 8;   // int32 flag words per split pair (ready + arrival count per 32-row quarter)
+struct AttnScratch {
+  unsigned* sched = nullptr;
+  int* flags = nullptr;
+  float* part = nullptr;
+  int cap_pairs = 0;
+};
+// bytes of flags + partials that never limit the split of a (B, T, H) problem
+size_t attention_scratch_bytes(int B, int T, int H);
+cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, const AttnScratch* scratch,
+                                int* status, cudaStream_t s);
+cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C,
+                             const AttnScratch* scratch, int* status, cudaStream_t s);
 
 // ---- cross-entropy finalisation -------------------------------------------
 // token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
