@@ -75,15 +75,17 @@ struct TcLayout {
 __device__ __forceinline__ float bf2f(const bf16 v) { return __bfloat162float(v); }
 
 // Bias slice of one 32-column chunk (bf16 -> fp32 registers); zeros past N.
-__device__ __forceinline__ void load_bias32(const bf16* bias, int col0, int N, float (&b)[32]) {
+// The same 32 bias values as bf16 pairs (lo = even column), zero past N.
+__device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int N, uint32_t (&b)[16]) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     const int col = col0 + g * 8;
     uint4 w = make_uint4(0, 0, 0, 0);
     if (col < N) w = __ldg(reinterpret_cast<const uint4*>(bias + col));
-    const bf16* bb = reinterpret_cast<const bf16*>(&w);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) b[g * 8 + j] = bf2f(bb[j]);
+    b[4 * g] = w.x;
+    b[4 * g + 1] = w.y;
+    b[4 * g + 2] = w.z;
+    b[4 * g + 3] = w.w;
   }
 }
 
@@ -340,33 +342,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
       } else {
-        // bias / GELU / residual: one 32-column chunk at a time (TMEM load,
-        // bias, activation, swizzled staging, TMA store or reduce-add)
-#pragma unroll 1
+        // bias / GELU / residual, 32 columns at a time (bias, activation,
+        // swizzled staging, TMA store or reduce-add). The TMEM load and bias
+        // of chunk c+1 are in flight while chunk c is computed and stored, and
+        // the accumulator goes back to the MMA warp as soon as its last chunk
+        // is in registers.
+        const int nch = (row0 < M && nvalid > 0) ? min(L::CHUNKS, (nvalid + 31) / 32) : 0;   // warp-uniform
+        const bf16* bias_p = static_cast<const bf16*>(args.bias);
+        uint32_t v[2][32];
+        uint32_t braw[2][16];   // bias as bf16 pairs
+        if (nch > 0) {
+          tmem_ld_32x32b_x32(t_row, v[0]);
+          load_bias32_raw(bias_p, cbase, N, braw[0]);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+#pragma unroll
         for (int c = 0; c < L::CHUNKS; ++c) {
-          if (c * 32 >= nvalid || row0 >= M) break;   // warp-uniform: nothing of this warp's rows to write
+          if (c >= nch) break;
           const int col0 = cbase + c * 32;
-          float bias[32];
-          load_bias32(static_cast<const bf16*>(args.bias), col0, N, bias);
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
+          if (c + 1 < nch) {
+            tmem_ld_32x32b_x32(t_row + (c + 1) * 32, v[(c + 1) & 1]);
+            load_bias32_raw(bias_p, col0 + 32, N, braw[(c + 1) & 1]);
+          } else {   // the accumulator slice is all in registers: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+          }
+          const uint32_t* vc = v[c & 1];
+          const uint32_t* bc = braw[c & 1];
           uint32_t pk[32];
           if (EPI == EPI_RESID) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) pk[j] = __float_as_uint(__uint_as_float(v[j]) + bias[j]);
+            for (int j = 0; j < 16; ++j) {
+              pk[2 * j] = __float_as_uint(__uint_as_float(vc[2 * j]) + __uint_as_float(bc[j] << 16));
+              pk[2 * j + 1] = __float_as_uint(__uint_as_float(vc[2 * j + 1]) + __uint_as_float(bc[j] & 0xffff0000u));
+            }
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
+              const float b0 = __uint_as_float(bc[j] << 16), b1 = __uint_as_float(bc[j] & 0xffff0000u);
               if (EPI == EPI_GELU) {
-                uint64_t y2 = f2_add(f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])),
-                                     f2_pack(bias[2 * j], bias[2 * j + 1]));
+                uint64_t y2 = f2_add(f2_pack(__uint_as_float(vc[2 * j]), __uint_as_float(vc[2 * j + 1])), f2_pack(b0, b1));
                 y2 = gelu_erf_x2(y2);
                 float a, b;
                 f2_unpack(y2, a, b);
                 pk[j] = pack_bf16x2(a, b);
               } else {
-                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) + bias[2 * j], __uint_as_float(v[2 * j + 1]) + bias[2 * j + 1]);
+                pk[j] = pack_bf16x2(__uint_as_float(vc[2 * j]) + b0, __uint_as_float(vc[2 * j + 1]) + b1);
               }
             }
           }
@@ -398,10 +424,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           store_pending = true;
         }
-        // Accumulator fully read: hand it back to the MMA warp.
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
       }
     }
     if (EPI != EPI_LMHEAD && lane == 0) bulk_wait_all();
