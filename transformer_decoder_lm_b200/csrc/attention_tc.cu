@@ -519,6 +519,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         continue;
       }
       float fa = 0.f, fb = 1.f / l;
+      bool own_first = false;
       const float* pb = part + (size_t)w.pair * ATTN_PART_FLOATS;
       if (kSplit && merge) {   // merge with the other half's partial rows
         bool got = true;
@@ -529,12 +530,17 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
           ok = false;
           break;
         }
-        const float m1 = __ldcg(pb + PART_M + r), l1 = __ldcg(pb + PART_L + r);
-        const float mx = fmaxf(m1, m);
-        const float a1 = ex2_approx(m1 - mx), a2 = ex2_approx(m - mx);
-        const float inv = 1.f / (l1 * a1 + l * a2);
-        fa = a1 * inv;
-        fb = a2 * inv;
+        // the same arithmetic whichever half merges: (1) is always the key
+        // range [0, a), (2) the range holding the diagonal
+        const float mo = __ldcg(pb + PART_M + r), lo = __ldcg(pb + PART_L + r);
+        own_first = w.role == ROLE_FIRST;
+        const float m1 = own_first ? m : mo, l1 = own_first ? l : lo;
+        const float m2 = own_first ? mo : m, l2 = own_first ? lo : l;
+        const float mx = fmaxf(m1, m2);
+        const float a1 = ex2_approx(m1 - mx), a2 = ex2_approx(m2 - mx);
+        const float inv = 1.f / (l1 * a1 + l2 * a2);
+        fa = a1 * inv;   // factor of range (1)
+        fb = a2 * inv;   // factor of range (2)
       }
       uint32_t pk[32];
 #pragma unroll
@@ -543,17 +549,21 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         tmem_ld_32x32b_x32(tO + c * 32, o);
         tmem_ld_wait();
         float v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * fb;
-        if (kSplit && merge) {
+        if (kSplit && merge) {   // y = O1 fa + O2 fb, rounded the same way whichever half holds O1
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const float4 q = __ldcg(reinterpret_cast<const float4*>(pb) + (c * 8 + u) * 128 + r);
-            v[4 * u] = fmaf(q.x, fa, v[4 * u]);
-            v[4 * u + 1] = fmaf(q.y, fa, v[4 * u + 1]);
-            v[4 * u + 2] = fmaf(q.z, fa, v[4 * u + 2]);
-            v[4 * u + 3] = fmaf(q.w, fa, v[4 * u + 3]);
+            const float qo[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float own = __uint_as_float(o[4 * u + k]);
+              const float o1 = own_first ? own : qo[k], o2 = own_first ? qo[k] : own;
+              v[4 * u + k] = fmaf(o1, fa, o2 * fb);
+            }
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * fb;
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[c * 16 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
