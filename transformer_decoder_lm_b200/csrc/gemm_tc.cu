@@ -7,15 +7,15 @@
 // with fp32 accumulation, A [M, K] and B [N, K] both K-major (the
 // nn.Linear [out, in] layout is already the K-major B operand).
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 2 + BN/16 warps):
 //   warp 0      TMA producer: 128x64 A box and BNx64 B box per stage, 128-byte
 //               swizzle, 4-deep ring of shared-memory stages.
 //   warp 1      allocates 2*BN TMEM columns and issues tcgen05.mma
 //               (M=128, N=BN, K=16, four per 64-wide k-block) into one of two
 //               TMEM accumulators; tcgen05.commit frees smem stages and hands
 //               finished accumulators to the epilogue.
-//   warps 2..9  epilogue, two warps per TMEM lane quadrant (rows), each taking
-//               half of the tile's columns, 32 columns per tcgen05.ld:
+//   warps 2..   epilogue, one warp per TMEM lane quadrant (32 rows) and
+//               64-column group (BN/16 warps), 32 columns per tcgen05.ld:
 //                 EPI_BIAS / EPI_GELU  +bias (+GELU erf), bf16, staged in
 //                                      64B-swizzled smem, TMA store;
 //                 EPI_RESID            +bias, fp32, staged in 128B-swizzled
@@ -30,7 +30,7 @@
 // main loop of tile i+1. Tiles are walked M-fastest so that concurrently
 // running CTAs share B tiles in L2 (the 77 MB wte is streamed ~once).
 //
-// The lm_head epilogue never needs the logits in HBM: per row and half tile
+// The lm_head epilogue never needs the logits in HBM: per row and 64-column group
 // it emits (max, sum exp(z - max)) and, where the target column lies, the
 // target logit; ce.cu finishes the log-sum-exp. Columns at or past N (the
 // vocabulary padded up to the tile width by TMA zero fill) are excluded from
@@ -52,24 +52,30 @@ namespace g2 {
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
 constexpr int TC_STAGES = 4;
-constexpr int TC_EPI_WARPS = 8;
-constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
-constexpr int STAGE_BUF_BYTES = 4096;   // per epilogue warp: 32 rows x 128 B
-
-template <int BN>
+template <int BN, int EPI>
 struct TcLayout {
+  // Each epilogue warp owns 32 rows (one TMEM lane quadrant) x COLS_PER_WARP
+  // columns: 64 (BN / 16 warps), or half the tile (8 warps; BN = 128, 256) for the lm_head
+  // without logits, whose epilogue has slack and whose warps would only
+  // compete with the MMA issuer.
+  static constexpr int COLS_PER_WARP = (EPI == EPI_LMHEAD && BN % 128 == 0) ? BN / 2 : 64;
+  static constexpr int EPI_WARPS = 4 * (BN / COLS_PER_WARP);
+  static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+  // per epilogue warp: one 32 x 32 chunk (bf16: 2 KB, fp32 residual: 4 KB),
+  // or 8 logits rows x 64 fp32 (2 KB)
+  static constexpr int STAGE_BUF_BYTES = EPI == EPI_RESID ? 4096 : 2048;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int EPI_OFFSET = TC_STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFFSET = EPI_OFFSET + TC_EPI_WARPS * STAGE_BUF_BYTES;
+  static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_WARPS * STAGE_BUF_BYTES;
   static constexpr int NUM_BARS = 2 * TC_STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
   static constexpr int SMEM_BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;   // + holders, 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
-  static constexpr int COLS_PER_WARP = BN / 2;
   static constexpr int CHUNKS = COLS_PER_WARP / 32;
+  static constexpr int GROUPS = BN / 64;   // lm_head: 64-column log-sum-exp groups per tile
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(COLS_PER_WARP % 32 == 0, "epilogue chunks are 32 columns");
+  static_assert(BN % COLS_PER_WARP == 0 && COLS_PER_WARP % 64 == 0, "whole 64-column groups per warp");
 };
 
 __device__ __forceinline__ float bf2f(const bf16 v) { return __bfloat162float(v); }
@@ -90,10 +96,11 @@ __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int 
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
-  using L = TcLayout<BN>;
+  using L = TcLayout<BN, EPI>;
+  constexpr bool kLM = EPI == EPI_LMHEAD || EPI == EPI_LMHEAD_LOGITS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
@@ -119,7 +126,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], TC_EPI_WARPS);
+      mbar_init(&tempty[b], L::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -128,7 +135,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (EPI != EPI_LMHEAD) tma_prefetch_desc(&tmC);
+    if (!kLM) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, L::TMEM_COLS);
@@ -226,8 +233,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quadrant = rows q*32 .. q*32+31
-    const int half = (warp - 2) >> 2;        // which half of the tile's columns
-    uint8_t* sbuf = smem + L::EPI_OFFSET + (warp - 2) * STAGE_BUF_BYTES;
+    const int cg = (warp - 2) >> 2;          // which 64-column group of the tile
+    uint8_t* sbuf = smem + L::EPI_OFFSET + (warp - 2) * L::STAGE_BUF_BYTES;
     const uint32_t sb = smem_u32(sbuf);
     constexpr float LOG2E = 1.4426950408889634f;
     bool store_pending = false;
@@ -240,10 +247,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int row0 = m0 + q * 32;          // first row of this warp
       const int row = row0 + lane;
       const bool row_ok = row < M;
-      const int cbase = n0 + half * L::COLS_PER_WARP;
+      const int cbase = n0 + cg * L::COLS_PER_WARP;
       const int nvalid = min(L::COLS_PER_WARP, N - cbase);   // may be <= 0 (warp-uniform)
       int tgt = -1;
-      if (EPI == EPI_LMHEAD) tgt = (row_ok && args.targets != nullptr) ? args.targets[row] : -1;
+      if (kLM) tgt = (row_ok && args.targets != nullptr) ? args.targets[row] : -1;
 
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
         if (lane == 0) {
@@ -253,11 +260,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * L::COLS_PER_WARP;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + cg * L::COLS_PER_WARP;
       // lm_head: pull this warp's whole slice of the accumulator into registers
       // with a single wait and give the TMEM buffer back before any arithmetic.
-      uint32_t r[EPI == EPI_LMHEAD ? L::CHUNKS : 1][32];
-      if (EPI == EPI_LMHEAD) {
+      uint32_t r[kLM ? L::CHUNKS : 1][32];
+      if (kLM) {
 #pragma unroll
         for (int c = 0; c < L::CHUNKS; ++c)
           if (c * 32 < nvalid) tmem_ld_32x32b_x32(t_row + c * 32, r[c]);
@@ -267,28 +274,40 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0) mbar_arrive(&tempty[acc]);
       }
 
-      if (EPI == EPI_LMHEAD) {
-        // log-sum-exp partial of this row over the valid columns of the half tile
-        // 8 independent partial maxima / sums keep the dependency chains short;
-        // columns at or past N count as -inf (exp2 gives 0)
-        float pm[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) pm[j] = -INFINITY;
+      if (kLM) {
+        // log-sum-exp partials of this row, one per 64-column group (the
+        // same arithmetic whichever warp layout runs, so the losses do not
+        // depend on whether logits are written): 8 independent partial
+        // maxima / sums keep the dependency chains short; columns at or past
+        // N count as -inf (exp2 gives 0)
 #pragma unroll
         for (int c = 0; c < L::CHUNKS; ++c)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 32; ++j)
             if (c * 32 + j >= nvalid) r[c][j] = __float_as_uint(-INFINITY);
-            pm[j & 7] = fmaxf(pm[j & 7], __uint_as_float(r[c][j]));
-          }
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        const float nm2 = mx * LOG2E;
-        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < L::CHUNKS; ++c)
+        for (int gi = 0; gi < L::CHUNKS / 2; ++gi) {
+          float pm[8];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) ps[j & 7] += ex2_approx(fmaf(__uint_as_float(r[c][j]), LOG2E, -nm2));
-        const float s0 = ps[0] + ps[1], s1 = ps[2] + ps[3], s2 = ps[4] + ps[5], s3 = ps[6] + ps[7];
+          for (int j = 0; j < 8; ++j) pm[j] = -INFINITY;
+#pragma unroll
+          for (int c = 2 * gi; c < 2 * gi + 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pm[j & 7] = fmaxf(pm[j & 7], __uint_as_float(r[c][j]));
+          const float mx =
+              fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+          const float nm2 = mx * LOG2E;
+          float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 2 * gi; c < 2 * gi + 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ps[j & 7] += ex2_approx(fmaf(__uint_as_float(r[c][j]), LOG2E, -nm2));
+          const float s0 = ps[0] + ps[1], s1 = ps[2] + ps[3], s2 = ps[4] + ps[5], s3 = ps[6] + ps[7];
+          // rows of `part` are the 64-column groups of the vocabulary
+          if (row_ok)
+            args.part[(size_t)(n_blk * L::GROUPS + cg * (L::CHUNKS / 2) + gi) * M + row] =
+                gi * 64 < nvalid ? make_float2(mx, (s0 + s1) + (s2 + s3)) : make_float2(-INFINITY, 0.f);
+        }
         const int tj = tgt - cbase;
         float tgt_val = 0.f;
 #pragma unroll
@@ -300,22 +319,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (mine && tj == c * 32 + j) tgt_val = __uint_as_float(r[c][j]);
           }
         }
-        if (nvalid > 0 && row_ok) {
-          // one partial per (row, half tile): rows of `part` are column groups of BN/2
-          args.part[(size_t)(n_blk * 2 + half) * M + row] = make_float2(mx, (s0 + s1) + (s2 + s3));
-          if (tj >= 0 && tj < nvalid) args.tgt_logit[row] = tgt_val;
-        } else if (row_ok) {
-          args.part[(size_t)(n_blk * 2 + half) * M + row] = make_float2(-INFINITY, 0.f);
-        }
-        if (args.out != nullptr) {
+        if (row_ok && tj >= 0 && tj < nvalid) args.tgt_logit[row] = tgt_val;
+        if (EPI == EPI_LMHEAD_LOGITS) {
           // fp32 logits. The row pitch V is odd, so rows are only 4-byte
           // aligned and neither vector nor TMA stores apply; short unaligned
           // row pieces leave partial 32-byte sectors that write slowly. So
-          // each row's 128 columns leave as one contiguous 512-byte run:
-          // 8 rows at a time are transposed through this warp's 4 KB of
-          // shared memory (row rr at rr * 512, 16-byte unit u stored at
+          // each row's 64 columns leave as one contiguous 256-byte run:
+          // 8 rows at a time are transposed through this warp's 2 KB of
+          // shared memory (row rr at rr * 256, 16-byte unit u stored at
           // unit u ^ rr, conflict-free both ways) and written by all 32 lanes
-          // as four back-to-back 128-byte stores per row.
+          // as two back-to-back 128-byte stores per row.
           float* lg = static_cast<float*>(args.out);
 #pragma unroll 1
           for (int g = 0; g < 4; ++g) {
@@ -323,7 +336,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const int rr = lane & 7;
 #pragma unroll
               for (int u = 0; u < 8 * L::CHUNKS; ++u)
-                st_shared_v4(sb + rr * 512 + ((u ^ rr) << 4), r[u >> 3][4 * (u & 7)], r[u >> 3][4 * (u & 7) + 1],
+                st_shared_v4(sb + rr * 256 + ((u ^ rr) << 4), r[u >> 3][4 * (u & 7)], r[u >> 3][4 * (u & 7) + 1],
                              r[u >> 3][4 * (u & 7) + 2], r[u >> 3][4 * (u & 7) + 3]);
             }
             __syncwarp();
@@ -334,65 +347,53 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
               for (int k = 0; k < L::CHUNKS; ++k) {
                 const int e = 32 * k + lane;
-                const float val = ld_shared_f32(sb + rr * 512 + (((8 * k + (lane >> 2)) ^ rr) << 4) + ((lane & 3) << 2));
-                if (grow < M && e < nvalid) dst[e] = val;
+                const float val = ld_shared_f32(sb + rr * 256 + (((8 * k + (lane >> 2)) ^ rr) << 4) + ((lane & 3) << 2));
+                if (grow < M && e < nvalid) __stcs(dst + e, val);   // streaming: evict first from L2
               }
             }
             __syncwarp();
           }
         }
       } else {
-        // bias / GELU / residual, 32 columns at a time (bias, activation,
-        // swizzled staging, TMA store or reduce-add). The TMEM load and bias
-        // of chunk c+1 are in flight while chunk c is computed and stored, and
-        // the accumulator goes back to the MMA warp as soon as its last chunk
-        // is in registers.
+        // bias / GELU / residual: both 32-column chunks of this warp's slice
+        // come out of TMEM with one wait and the accumulator goes straight
+        // back to the MMA warp; then per chunk: bias, activation, swizzled
+        // staging, TMA store or reduce-add.
         const int nch = (row0 < M && nvalid > 0) ? min(L::CHUNKS, (nvalid + 31) / 32) : 0;   // warp-uniform
+        uint32_t v[L::CHUNKS][32];
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c)
+          if (c < nch) tmem_ld_32x32b_x32(t_row + c * 32, v[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
         const bf16* bias_p = static_cast<const bf16*>(args.bias);
-        uint32_t v[2][32];
-        uint32_t braw[2][16];   // bias as bf16 pairs
-        if (nch > 0) {
-          tmem_ld_32x32b_x32(t_row, v[0]);
-          load_bias32_raw(bias_p, cbase, N, braw[0]);
-        } else {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
-        }
 #pragma unroll
         for (int c = 0; c < L::CHUNKS; ++c) {
           if (c >= nch) break;
           const int col0 = cbase + c * 32;
-          tmem_ld_wait();
-          if (c + 1 < nch) {
-            tmem_ld_32x32b_x32(t_row + (c + 1) * 32, v[(c + 1) & 1]);
-            load_bias32_raw(bias_p, col0 + 32, N, braw[(c + 1) & 1]);
-          } else {   // the accumulator slice is all in registers: hand it back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
-          }
-          const uint32_t* vc = v[c & 1];
-          const uint32_t* bc = braw[c & 1];
-          uint32_t pk[32];
+          uint32_t bc[16];   // bias as bf16 pairs
+          load_bias32_raw(bias_p, col0, N, bc);
+          uint32_t* pk = v[c];   // results overwrite the accumulator values in place
           if (EPI == EPI_RESID) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              pk[2 * j] = __float_as_uint(__uint_as_float(vc[2 * j]) + __uint_as_float(bc[j] << 16));
-              pk[2 * j + 1] = __float_as_uint(__uint_as_float(vc[2 * j + 1]) + __uint_as_float(bc[j] & 0xffff0000u));
+              pk[2 * j] = __float_as_uint(__uint_as_float(v[c][2 * j]) + __uint_as_float(bc[j] << 16));
+              pk[2 * j + 1] = __float_as_uint(__uint_as_float(v[c][2 * j + 1]) + __uint_as_float(bc[j] & 0xffff0000u));
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const float b0 = __uint_as_float(bc[j] << 16), b1 = __uint_as_float(bc[j] & 0xffff0000u);
+              const float x0 = __uint_as_float(v[c][2 * j]), x1 = __uint_as_float(v[c][2 * j + 1]);
               if (EPI == EPI_GELU) {
-                uint64_t y2 = f2_add(f2_pack(__uint_as_float(vc[2 * j]), __uint_as_float(vc[2 * j + 1])), f2_pack(b0, b1));
-                y2 = gelu_erf_x2(y2);
+                const uint64_t y2 = gelu_erf_x2(f2_add(f2_pack(x0, x1), f2_pack(b0, b1)));
                 float a, b;
                 f2_unpack(y2, a, b);
                 pk[j] = pack_bf16x2(a, b);
               } else {
-                pk[j] = pack_bf16x2(__uint_as_float(vc[2 * j]) + b0, __uint_as_float(vc[2 * j + 1]) + b1);
+                pk[j] = pack_bf16x2(x0 + b0, x1 + b1);
               }
             }
           }
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
     }
-    if (EPI != EPI_LMHEAD && lane == 0) bulk_wait_all();
+    if (!kLM && lane == 0) bulk_wait_all();
     __syncwarp();
   }
 
@@ -467,20 +468,33 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
   return r == CUDA_SUCCESS;
 }
 
+
+// The residual epilogue's 4 KB staging per warp does not fit next to the ring
+// at BN = 256 (gemm_tc_pick_bn never picks it there).
+template <int BN, int EPI>
+constexpr bool tc_supported() {
+  return !(EPI == EPI_RESID && BN == 256);
+}
+
 template <int BN, int EPI>
 cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC, const GemmArgs& a,
                        int num_sms, cudaStream_t s) {
-  using L = TcLayout<BN>;
-  const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
-  const int grid = std::min(tiles, num_sms);
-  if (grid <= 0) return cudaSuccess;
-  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(TC_THREADS), L::SMEM_BYTES, s, tA, tB, tC, a);
+  if constexpr (!tc_supported<BN, EPI>()) {
+    return cudaErrorInvalidValue;
+  } else {
+    using L = TcLayout<BN, EPI>;
+    const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
+    const int grid = std::min(tiles, num_sms);
+    if (grid <= 0) return cudaSuccess;
+    return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, tA, tB, tC, a);
+  }
 }
 
 template <int BN, int EPI>
 cudaError_t set_attr_one() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcLayout<BN>::SMEM_BYTES);
+  if constexpr (!tc_supported<BN, EPI>()) return cudaSuccess;
+  else return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcLayout<BN, EPI>::SMEM_BYTES);
 }
 
 template <int BN>
@@ -490,7 +504,9 @@ cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, con
     case EPI_BIAS: return launch_one<BN, EPI_BIAS>(tA, tB, tC, a, num_sms, s);
     case EPI_GELU: return launch_one<BN, EPI_GELU>(tA, tB, tC, a, num_sms, s);
     case EPI_RESID: return launch_one<BN, EPI_RESID>(tA, tB, tC, a, num_sms, s);
-    case EPI_LMHEAD: return launch_one<BN, EPI_LMHEAD>(tA, tB, tC, a, num_sms, s);
+    case EPI_LMHEAD:
+      return a.out != nullptr ? launch_one<BN, EPI_LMHEAD_LOGITS>(tA, tB, tC, a, num_sms, s)
+                              : launch_one<BN, EPI_LMHEAD>(tA, tB, tC, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -524,14 +540,16 @@ bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-int gemm_tc_n_tiles(int N, int bn) { return 2 * ((N + bn - 1) / bn); }
+int gemm_tc_n_tiles(int N, int bn) { return (bn / 64) * ((N + bn - 1) / bn); }   // TcLayout::GROUPS per tile
 
-int gemm_tc_pick_bn(int M, int N, int num_sms) {
+int gemm_tc_pick_bn(int M, int N, int num_sms, int epi) {
+  // The residual epilogue runs with tiles of at most 192 columns.
+  const int max_bn = epi == EPI_RESID ? 192 : 256;
   // G2_GEMM_BN=64|128|192|256 pins the tile width (tests use it to cover
   // every instantiation); otherwise the width is chosen by the cost model below.
   if (const char* e = getenv("G2_GEMM_BN")) {
     const int v = atoi(e);
-    if (v == 64 || v == 128 || v == 192 || v == 256) return v;
+    if (v == 64 || v == 128 || v == 192 || v == 256) return v < max_bn ? v : max_bn;
   }
   // Estimated cost = waves x per-tile cost. Narrower tiles re-read A from
   // shared memory more often per FLOP (the 128-row MMA at N=128 runs at
@@ -541,9 +559,10 @@ int gemm_tc_pick_bn(int M, int N, int num_sms) {
   const int cand[4] = {256, 192, 128, 64};
   const double unit[4] = {256.0, 192.0, 200.0, 150.0};
   const int mt = (M + TC_BM - 1) / TC_BM;
-  int best = 256;
+  int best = max_bn;
   double best_cost = 1e30;
   for (int i = 0; i < 4; ++i) {
+    if (cand[i] > max_bn) continue;
     const long tiles = (long)mt * ((N + cand[i] - 1) / cand[i]);
     const long waves = (tiles + num_sms - 1) / num_sms;
     const double cost = waves * unit[i];
@@ -572,7 +591,8 @@ cudaError_t gemm_tc_set_attributes() {
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_BIAS>();        \
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU>();        \
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID>();       \
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD>();      \
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD_LOGITS>();
   G2_ATTR(256)
   G2_ATTR(192)
   G2_ATTR(128)

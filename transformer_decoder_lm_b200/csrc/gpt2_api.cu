@@ -36,9 +36,6 @@ inline int bn_index(int bn) { return bn == 256 ? 0 : (bn == 192 ? 1 : (bn == 128
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// lm_head partials per row: two column groups per tile of width >= 128 (tcgen05
-// path) or one per 64-column tile (SIMT path); both fit in 2 * ceil(V / 128).
-inline size_t lmhead_groups(int V) { return 2 * (size_t)((V + LMHEAD_MIN_BN - 1) / LMHEAD_MIN_BN); }
 
 struct LayerPtrs {
   const void *ln1_g, *ln1_b, *attn_w, *attn_b, *attn_proj_w, *attn_proj_b;
@@ -58,7 +55,7 @@ Plan plan_workspace(const gpt2_config_t& c, int max_B, int max_T) {
   const long M = (long)max_B * max_T;
   const size_t es = c.dtype == GPT2_BF16 ? 2 : 4;
   const size_t C = (size_t)c.n_embd;
-  const size_t n_tiles = lmhead_groups(c.vocab);
+  const size_t n_tiles = lmhead_groups_max(c.vocab);
   Plan p;
   size_t o = 0;
   p.x = o;      o += align256(M * C * 4);
@@ -160,7 +157,7 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   a.status = m->status;
   cudaError_t e;
   if (m->bf16) {
-    const int bn = gemm_tc_pick_bn(M, N, m->num_sms);
+    const int bn = gemm_tc_pick_bn(M, N, m->num_sms, epi);
     e = gemm_tc_launch(epi, bn, *tmA, wmaps[bn_index(bn)], *tmC, a, m->num_sms, s);
   } else {
     e = gemm_simt_launch(epi, static_cast<const float*>(A), static_cast<const float*>(W), a, s);
@@ -230,7 +227,7 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     int n_tiles;
     if (m->ev_lm_begin) G2_CK(cudaEventRecord(m->ev_lm_begin, s));
     if (m->bf16) {
-      const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms), LMHEAD_MIN_BN);
+      const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
       n_tiles = gemm_tc_n_tiles(V, bn);
       G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, tm_h, m->wte_map[bn_index(bn)], tm_h, a, m->num_sms, s));
     } else {
@@ -464,7 +461,7 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
   int sms = 0;
   int rc = device_setup(nullptr, &sms);
   if (rc != GPT2_OK) return rc;
-  const int bn = gemm_tc_pick_bn(M, N, sms);
+  const int bn = gemm_tc_pick_bn(M, N, sms, epilogue);
   CUtensorMap ta, tb, tc;
   if (!make_tmap_bf16(&ta, A, M, K, K, 128) || !make_tmap_bf16(&tb, W, N, K, K, bn)) return GPT2_ERR_CUDA;
   const bool ok_c = epilogue == GPT2_EPI_BIAS_RESID ? make_tmap_out_f32(&tc, out, M, N, N)
@@ -487,7 +484,7 @@ int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, vo
 
 size_t gpt2_op_lmhead_ce_workspace_bytes(int dtype, int M, int V) {
   if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || M < 1 || V < 1) return 0;
-  return align256(lmhead_groups(V) * (size_t)M * sizeof(float2)) + 2 * align256((size_t)M * 4);
+  return align256(lmhead_groups_max(V) * (size_t)M * sizeof(float2)) + 2 * align256((size_t)M * 4);
 }
 
 int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t* targets, int M, int C, int V,
@@ -499,7 +496,7 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
   if (ws_bytes < gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V)) return GPT2_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t n_tiles_max = lmhead_groups(V);
+  const size_t n_tiles_max = lmhead_groups_max(V);
   float2* part = reinterpret_cast<float2*>(ws);
   float* tgt = reinterpret_cast<float*>(ws + align256(n_tiles_max * (size_t)M * sizeof(float2)));
   float* tok = tgt + align256((size_t)M * 4) / 4;
@@ -519,7 +516,7 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
     int sms = 0;
     int rc = device_setup(nullptr, &sms);
     if (rc != GPT2_OK) return rc;
-    const int bn = std::max(gemm_tc_pick_bn(M, V, sms), LMHEAD_MIN_BN);
+    const int bn = std::max(gemm_tc_pick_bn(M, V, sms, EPI_LMHEAD), LMHEAD_MIN_BN);
     n_tiles = gemm_tc_n_tiles(V, bn);
     CUtensorMap ta, tb;
     if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;

@@ -27,7 +27,9 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 
 // Epilogues of the Linear layers (values match the public GPT2_EPI_*),
 // plus the fused lm_head / cross-entropy epilogue.
-enum EpiKind : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_LMHEAD = 3 };
+// EPI_LMHEAD_LOGITS is the lm_head kernel that also writes the logits;
+// gemm_tc_launch picks it for EPI_LMHEAD when GemmArgs::out is set.
+enum EpiKind : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_LMHEAD = 3, EPI_LMHEAD_LOGITS = 4 };
 
 struct GemmArgs {
   int M, N, K;
@@ -58,12 +60,16 @@ bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t 
 int gemm_tc_n_tiles(int N, int bn);
 // The lm_head runs with tiles of at least this width.
 constexpr int LMHEAD_MIN_BN = 128;
+// lm_head partials per row: one per 64-column group of a tcgen05 tile (tiles
+// of BN columns cover V padded up to a multiple of BN) or per 64-column SIMT
+// tile; at most ceil(V / 64) + 3 either way.
+inline size_t lmhead_groups_max(int V) { return (size_t)((V + 63) / 64) + 3; }
 
 // ---- tcgen05 GEMM (bf16) -------------------------------------------------
 // C = A[M,K] . B[N,K]^T with the epilogue `epi`. K % 64 == 0, N % 8 == 0.
 // tmA: box 128 x 64 over A; tmB: box BN x 64 over B, BN from gemm_tc_pick_bn;
 // tmC: the output map (make_tmap_out_*; unused by EPI_LMHEAD).
-int gemm_tc_pick_bn(int M, int N, int num_sms);
+int gemm_tc_pick_bn(int M, int N, int num_sms, int epi);
 cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
                            const GemmArgs& a, int num_sms, cudaStream_t s);
 cudaError_t gemm_tc_set_attributes();

@@ -76,7 +76,7 @@ extern "C" int gpt2_op_lmhead_ce_noalloc(int dtype, const void* hf, const void* 
   if (dtype == GPT2_BF16 && (C % 64)) return GPT2_ERR_UNSUPPORTED;
   // Same scratch layout as gpt2_op_lmhead_ce: partials [groups][M] float2,
   // target logits [M], per-position losses [M].
-  const size_t groups = 2 * (size_t)((V + LMHEAD_MIN_BN - 1) / LMHEAD_MIN_BN);
+  const size_t groups = lmhead_groups_max(V);
   const size_t part_bytes = align256(groups * (size_t)M * sizeof(float2));
   const size_t need = part_bytes + 2 * align256((size_t)M * 4);
   if (need > (size_t)GPT2_NOALLOC_SCRATCH_BYTES) return GPT2_ERR_SCRATCH_LIMIT;
@@ -102,7 +102,7 @@ extern "C" int gpt2_op_lmhead_ce_noalloc(int dtype, const void* hf, const void* 
   a.status = status;
   int n_groups;
   if (dtype == GPT2_BF16) {
-    const int bn = gemm_tc_pick_bn(M, V, d->num_sms) < LMHEAD_MIN_BN ? LMHEAD_MIN_BN : gemm_tc_pick_bn(M, V, d->num_sms);
+    const int bn = gemm_tc_pick_bn(M, V, d->num_sms, EPI_LMHEAD) < LMHEAD_MIN_BN ? LMHEAD_MIN_BN : gemm_tc_pick_bn(M, V, d->num_sms, EPI_LMHEAD);
     n_groups = gemm_tc_n_tiles(V, bn);
     CUtensorMap ta, tb;
     if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;
