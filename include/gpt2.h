@@ -216,7 +216,7 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
  * array of GPT2_NOALLOC_SCRATCH_BYTES inside this library, held on every GPU
  * that loads the library until the process exits. A call needs
  * gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V) of it (about
- * 16 * ceil(V / 128) bytes per row; V = 50257 allows up to 5335 rows); larger
+ * 8 * (ceil(V / 64) + 4) bytes per row; V = 50257 allows up to 5309 rows); larger
  * requests return GPT2_ERR_SCRATCH_LIMIT before any launch. The first call
  * on each device performs a one-time set-up there (it looks up the array's
  * device address, reads the SM count and sets kernel attributes), so make

@@ -15,48 +15,61 @@
 namespace g2 {
 
 // One block per 32 rows: lane = row, so every load of a partial is a
-// coalesced 256-byte read of one column group for 32 consecutive rows; the 8
-// warps take the column groups round-robin and their running (max, sum) pairs
-// are merged through shared memory.
-__global__ void __launch_bounds__(256) ce_rows_kernel(const float2* __restrict__ part, int n_tiles,
-                                                      const float* __restrict__ tgt_logit,
-                                                      const int* __restrict__ targets, int M, int V,
-                                                      float* __restrict__ token_loss, int* status) {
-  __shared__ float sm_m[8][32], sm_s[8][32];
+// coalesced 256-byte read of one column group for 32 consecutive rows. The 16
+// warps take the column groups round-robin, each warp with 4 independent
+// running (max, sum) pairs (groups 16 a + warp for a = j mod 4) so that the
+// merge chains overlap; the pairs are merged in a fixed order, per warp and
+// then across warps through shared memory (deterministic). Rescaling uses
+// exp(d) = 2^(d log2 e) on the SFU.
+constexpr int CE_WARPS = 16;
+
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  if (m2 == -INFINITY) return;   // a column group with no valid column
+  const float mn = fmaxf(m, m2);
+  s = s * ex2_approx((m - mn) * 1.4426950408889634f) + s2 * ex2_approx((m2 - mn) * 1.4426950408889634f);
+  m = mn;
+}
+
+__global__ void __launch_bounds__(32 * CE_WARPS) ce_rows_kernel(const float2* __restrict__ part, int n_tiles,
+                                                               const float* __restrict__ tgt_logit,
+                                                               const int* __restrict__ targets, int M, int V,
+                                                               float* __restrict__ token_loss, int* status) {
+  __shared__ float sm_m[CE_WARPS][32], sm_s[CE_WARPS][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 32 + lane;
   pdl_wait();
   pdl_trigger();
-  float m = -INFINITY, s = 0.f;
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, s[4] = {0.f, 0.f, 0.f, 0.f};
   if (row < M) {
-    for (int i = warp; i < n_tiles; i += 8) {
+    int i = warp;
+    for (; i + 3 * CE_WARPS < n_tiles; i += 4 * CE_WARPS) {
+      float2 p[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) p[a] = part[(size_t)(i + a * CE_WARPS) * M + row];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) lse_merge(m[a], s[a], p[a].x, p[a].y);
+    }
+    for (int a = 0; i < n_tiles; i += CE_WARPS, ++a) {
       const float2 p = part[(size_t)i * M + row];
-      if (p.x == -INFINITY) continue;   // a column group with no valid column
-      const float mn = fmaxf(m, p.x);
-      s = s * expf(m - mn) + p.y * expf(p.x - mn);
-      m = mn;
+      lse_merge(m[a], s[a], p.x, p.y);
     }
   }
-  sm_m[warp][lane] = m;
-  sm_s[warp][lane] = s;
+  lse_merge(m[0], s[0], m[1], s[1]);
+  lse_merge(m[2], s[2], m[3], s[3]);
+  lse_merge(m[0], s[0], m[2], s[2]);
+  sm_m[warp][lane] = m[0];
+  sm_s[warp][lane] = s[0];
   __syncthreads();
   if (warp == 0 && row < M) {
-    m = -INFINITY;
-    s = 0.f;
+    float mm = -INFINITY, ss = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const float m2 = sm_m[w][lane], s2 = sm_s[w][lane];
-      if (m2 == -INFINITY) continue;
-      const float mn = fmaxf(m, m2);
-      s = s * expf(m - mn) + s2 * expf(m2 - mn);
-      m = mn;
-    }
+    for (int w = 0; w < CE_WARPS; ++w) lse_merge(mm, ss, sm_m[w][lane], sm_s[w][lane]);
     const int tg = targets[row];
     float l = 0.f;
     if (tg >= V) {
       record_error(status, DEV_BAD_TOKEN);
     } else if (tg >= 0) {
-      l = (m + logf(s)) - tgt_logit[row];
+      l = (mm + logf(ss)) - tgt_logit[row];
     }
     token_loss[row] = l;
   }
@@ -112,7 +125,7 @@ __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__
 cudaError_t ce_finish_launch(const float2* part, int n_tiles, const float* tgt_logit, const int* targets, int M,
                              int V, float* token_loss, float* loss_out, int* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = launch_pdl(ce_rows_kernel, dim3((M + 31) / 32), dim3(256), 0, s, part, n_tiles, tgt_logit, targets,
+  cudaError_t e = launch_pdl(ce_rows_kernel, dim3((M + 31) / 32), dim3(32 * CE_WARPS), 0, s, part, n_tiles, tgt_logit, targets,
                              M, V, token_loss, status);
   if (e == cudaSuccess && loss_out)
     e = launch_pdl(ce_mean_kernel, dim3(1), dim3(1024), 0, s, token_loss, targets, M, V, loss_out, status);
