@@ -252,13 +252,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
-// One 32-bit column for 32 lanes (lane i of the warp <-> TMEM lane taddr.lane + i).
-__device__ __forceinline__ void tmem_st_32x32b_x1(uint32_t taddr, const uint32_t (&r)[1]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0]) : "memory");
-}
-__device__ __forceinline__ void tmem_ld_32x32b_x1(uint32_t taddr, uint32_t (&r)[1]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with a K-major A, an
@@ -290,24 +283,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 127 (inputs below -126 give about 2^-126): x = n + f
-// with n the nearest integer (by the 1.5 * 2^23 rounding trick) and
-// f in [-0.5, 0.5]; 2^f by a degree-4 polynomial fitted here for relative
-// error (max 2.7e-6 on that interval); 2^n added to the exponent field.
-// Used for a share of the softmax exponentials so that they do not all queue
-// on the SFU.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float fr = x - (t - 12582912.0f);
-  float p = fmaf(9.570068679749966e-3f, fr, 5.5917806923389435e-2f);
-  p = fmaf(p, fr, 2.40247443318367e-1f);
-  p = fmaf(p, fr, 6.931218504905701e-1f);
-  p = fmaf(p, fr, 9.999992847442627e-1f);
-  // low bits of t hold n (two's complement); shifting them into the exponent
-  // field is done in unsigned arithmetic (wrap-around is intended)
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
 
 // ---- packed fp32 pairs: on sm_100 one instruction adds, subtracts or
 // fuses-multiply-adds two floats held in a 64-bit register pair.
@@ -346,8 +321,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// ex2_poly on a pair of floats, the rounding split and the polynomial in
-// packed arithmetic (each lane the same IEEE operations as ex2_poly).
+// 2^x on the FMA pipe for a pair of floats in packed arithmetic, for
+// x <= 127 (inputs below -126 give about 2^-126): x = n + f with n the
+// nearest integer (by the 1.5 * 2^23 rounding trick) and f in [-0.5, 0.5];
+// 2^f by a degree-4 polynomial fitted here for relative error (max 2.7e-6 on
+// that interval); 2^n added to the exponent field (the low bits of t hold n
+// in two's complement; the shift into the exponent field wraps in unsigned
+// arithmetic, as intended). An alternative to the SFU for part of a softmax's
+// exponentials.
 __device__ __forceinline__ void ex2_poly_x2(uint64_t x, float& y0, float& y1) {
   float x0, x1;
   f2_unpack(x, x0, x1);
@@ -381,26 +362,9 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // With r = 1 / (...)^16 ~= erfc(|z|), 1 + erf(z) is 2 - r for z >= 0 and r
 // for z < 0 (no cancellation for negative inputs). Branch-free, one SFU
 // reciprocal; a huge |z| makes the power overflow to inf and r = 0.
-__device__ __forceinline__ float gelu_erf(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  float p = fmaf(z, 4.30638e-5f, 2.765672e-4f);
-  p = fmaf(z, p, 1.520143e-4f);
-  p = fmaf(z, p, 9.2705272e-3f);
-  p = fmaf(z, p, 4.22820123e-2f);
-  p = fmaf(z, p, 7.05230784e-2f);
-  p = fmaf(z, p, 1.0f);
-  p = p * p;   // ^2
-  p = p * p;   // ^4
-  p = p * p;   // ^8
-  p = p * p;   // ^16
-  const float r = rcp_approx(p);
-  const float one_plus_erf = x >= 0.f ? 2.0f - r : r;
-  return 0.5f * x * one_plus_erf;
-}
-
-// gelu_erf on a pair in packed fp32. With r = 1 - erf(|x|/sqrt2) from the
-// same approximation, gelu(x) = 0.5 x (1 + erf(x/sqrt2)) = relu(x) - 0.5 |x| r
-// for either sign of x (x >= 0: x - 0.5 x r; x < 0: 0.5 x r).
+// Computed here on a pair in packed fp32: with r = 1 - erf(|x|/sqrt2) as above,
+// gelu(x) = 0.5 x (1 + erf(x/sqrt2)) = relu(x) - 0.5 |x| r for either sign of
+// x (x >= 0: x - 0.5 x r; x < 0: 0.5 x r).
 __device__ __forceinline__ uint64_t gelu_erf_x2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);

@@ -78,8 +78,6 @@ struct TcLayout {
   static_assert(BN % COLS_PER_WARP == 0 && COLS_PER_WARP % 64 == 0, "whole 64-column groups per warp");
 };
 
-__device__ __forceinline__ float bf2f(const bf16 v) { return __bfloat162float(v); }
-
 // Bias slice of one 32-column chunk (bf16 -> fp32 registers); zeros past N.
 // The same 32 bias values as bf16 pairs (lo = even column), zero past N.
 __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int N, uint32_t (&b)[16]) {
