@@ -63,12 +63,21 @@ enum {
 
 /* Model shape. n_ctx is the size of the learned position table wpe
  * ("GPT-2 architecture analysis and implementation guide", section 1.2).
- * flags: reserved, must be 0. */
+ * flags: 0 or GPT2_FLAG_GELU_TANH; other bits must be 0. */
 typedef struct {
   int n_layer, n_head, n_embd, vocab, n_ctx;
   int dtype;          /* gpt2_dtype_t */
   unsigned flags;
 } gpt2_config_t;
+
+/* The MLP's activation is the tanh approximation
+ *   gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2 / pi) (x + 0.044715 x^3))),
+ * the form the pages attribute to the original GPT-2 ("Hand-writing GPT-2
+ * from scratch: the Transformer decoder core modules in PyTorch", section
+ * 3.4; "Reproducing GPT-2 124M", section 2.4), instead of the default exact
+ * erf form (F.gelu, "GPT-2 architecture analysis and implementation guide",
+ * section 2.2). */
+#define GPT2_FLAG_GELU_TANH 1u
 
 /* Weight pointers. wte [vocab, C] is also the lm_head weight (weight tying,
  * "Hand-writing GPT-2 from scratch ...", section 2.2 item 4). wpe [n_ctx, C].
@@ -177,14 +186,26 @@ int gpt2_op_layernorm(int dtype, const float* x, const void* g, const void* b,
                       int M, int C, void* out, void* stream);
 
 /* Linear layer y = A W^T + bias with A [M, K], W [N, K], bias [N], all of
- * `dtype`, and one of three epilogues:
- *   GPT2_EPI_BIAS        out [M, N] (`dtype`) = y
- *   GPT2_EPI_BIAS_GELU   out [M, N] (`dtype`) = gelu_erf(y)
- *   GPT2_EPI_BIAS_RESID  out fp32 [M, N] += y    (residual add in place)
+ * `dtype`, and one of four epilogues:
+ *   GPT2_EPI_BIAS             out [M, N] (`dtype`) = y
+ *   GPT2_EPI_BIAS_GELU        out [M, N] (`dtype`) = gelu_erf(y)
+ *   GPT2_EPI_BIAS_RESID       out fp32 [M, N] += y    (residual add in place)
+ *   GPT2_EPI_BIAS_GELU_TANH   out [M, N] (`dtype`) = gelu_tanh(y) (see GPT2_FLAG_GELU_TANH)
  * K and N must be multiples of 8 (bf16: K a multiple of 64). */
-enum { GPT2_EPI_BIAS = 0, GPT2_EPI_BIAS_GELU = 1, GPT2_EPI_BIAS_RESID = 2 };
+enum { GPT2_EPI_BIAS = 0, GPT2_EPI_BIAS_GELU = 1, GPT2_EPI_BIAS_RESID = 2, GPT2_EPI_BIAS_GELU_TANH = 3 };
 int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const void* bias,
                    int M, int N, int K, void* out, int* status, void* stream);
+
+/* Fixed sinusoidal position table ("Hand-writing GPT-2 from scratch: the
+ * Transformer decoder core modules in PyTorch", section 3.1, a variant the
+ * other pages do not use: they learn wpe): for pos in [0, n_ctx) and i in
+ * [0, C/2),
+ *   wpe[pos, 2i]     = sin(pos / 10000^(2i / C))
+ *   wpe[pos, 2i + 1] = cos(pos / 10000^(2i / C)),
+ * evaluated in double precision and rounded once to `dtype`. wpe is a device
+ * array [n_ctx, C] of `dtype`, C even; it can then be passed as the model's
+ * wpe. Returns GPT2_OK or an error code; asynchronous on `stream`. */
+int gpt2_fill_sinusoidal_wpe(int dtype, void* wpe, int n_ctx, int C, void* stream);
 
 /* Causal multi-head self-attention. qkv [B*T, 3C] (`dtype`, columns q | k | v,
  * head h at columns h*D..h*D+D-1 of each) -> y [B*T, C] (`dtype`), heads

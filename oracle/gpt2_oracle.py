@@ -6,8 +6,8 @@ path: only the tests, the smoke check and the bench's CPU-baseline leg may
 import it. It shares no code with the CUDA path; its only shared input is the
 seeded generator in ``synthetic``.
 
-Every step is the plain definition, with NumPy's matmul, exp, log and
-SciPy's erf as the only library primitives. There is no blocking, fusion or
+Every step is the plain definition, with NumPy's matmul, exp, log, tanh,
+sin, cos and SciPy's erf as the only library primitives. There is no blocking, fusion or
 reordering: attention materialises the full masked score matrix, the
 cross-entropy materialises the full logits.
 
@@ -54,10 +54,32 @@ def gelu(x: np.ndarray) -> np.ndarray:
     """Exact GELU, 0.5 x (1 + erf(x / sqrt 2)).
 
     [P3] section 2.2 applies F.gelu (the exact erf form); [P1] section 3.4
-    recommends approximate=False. The tanh form of [P4] section 2.4 is not
-    used.
+    recommends approximate=False. This is the default activation; gelu_tanh
+    is the flag-selected variant.
     """
     return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+
+
+def gelu_tanh(x: np.ndarray) -> np.ndarray:
+    """Tanh-approximation GELU, 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+
+    [P1] section 3.4 and [P4] section 2.4 give this form as the one of the
+    original GPT-2 implementation (the model's GPT2_FLAG_GELU_TANH variant).
+    """
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def sinusoidal_wpe(n_ctx: int, C: int) -> np.ndarray:
+    """Fixed sinusoidal position table [n_ctx, C] ([P1] section 3.1):
+    pe[pos, 2i] = sin(pos / 10000^(2i/C)), pe[pos, 2i+1] = cos(pos / 10000^(2i/C)),
+    pos from 0, i in [0, C/2)."""
+    pos = np.arange(n_ctx, dtype=np.float64)[:, None]
+    i = np.arange(C // 2, dtype=np.float64)[None, :]
+    angle = pos / np.power(10000.0, 2.0 * i / C)
+    pe = np.empty((n_ctx, C), dtype=np.float64)
+    pe[:, 0::2] = np.sin(angle)
+    pe[:, 1::2] = np.cos(angle)
+    return pe
 
 
 def linear(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray]) -> np.ndarray:
@@ -111,7 +133,8 @@ def causal_self_attention(qkv: np.ndarray, n_head: int, return_probs: bool = Fal
     return (out, probs) if return_probs else out
 
 
-def block(x: np.ndarray, lw: Dict[str, np.ndarray], n_head: int, eps: float = LN_EPS) -> np.ndarray:
+def block(x: np.ndarray, lw: Dict[str, np.ndarray], n_head: int, eps: float = LN_EPS,
+          act=None) -> np.ndarray:
     """One Pre-LN block: x += attn(ln_1(x)); x += mlp(ln_2(x)).
 
     [P1] section 3.2 (LN, attention, residual add, LN, MLP, residual add);
@@ -123,7 +146,7 @@ def block(x: np.ndarray, lw: Dict[str, np.ndarray], n_head: int, eps: float = LN
     y = causal_self_attention(qkv, n_head)
     x = x + linear(y, lw["attn_proj_w"], lw["attn_proj_b"])
     h = layer_norm(x, lw["ln2_g"], lw["ln2_b"], eps)
-    f = gelu(linear(h, lw["fc_w"], lw["fc_b"]))
+    f = (gelu if act is None else act)(linear(h, lw["fc_w"], lw["fc_b"]))
     x = x + linear(f, lw["mlp_proj_w"], lw["mlp_proj_b"])
     return x
 
@@ -143,21 +166,22 @@ def _as(d: Dict[str, np.ndarray], dtype) -> Dict[str, np.ndarray]:
 
 
 def hidden_states(weights: Dict[str, object], ids: np.ndarray, n_head: int,
-                  dtype=np.float64, eps: float = LN_EPS) -> np.ndarray:
+                  dtype=np.float64, eps: float = LN_EPS, act=None) -> np.ndarray:
     """Residual stream after every block, then ln_f: returns [B,T,C]
-    ([P1] section 4.1 forward steps 1-3)."""
+    ([P1] section 4.1 forward steps 1-3). `act` is the MLP activation
+    (None: gelu, the exact form)."""
     x = embed(weights, ids, dtype)
     for lw in weights["layers"]:
-        x = block(x, _as(lw, dtype), n_head, eps)
+        x = block(x, _as(lw, dtype), n_head, eps, act)
     return layer_norm(x, np.asarray(weights["lnf_g"], dtype), np.asarray(weights["lnf_b"], dtype), eps)
 
 
 def forward(weights: Dict[str, object], ids: np.ndarray, n_head: int,
-            dtype=np.float64, eps: float = LN_EPS) -> np.ndarray:
+            dtype=np.float64, eps: float = LN_EPS, act=None) -> np.ndarray:
     """Logits [B,T,V] = ln_f(x) wte^T, the lm_head tied to the token
     embedding with no bias ([P1] sections 2.2 and 4.1 step 4; [P4] section
     2.1 weight tying)."""
-    hf = hidden_states(weights, ids, n_head, dtype, eps)
+    hf = hidden_states(weights, ids, n_head, dtype, eps, act)
     return hf @ np.asarray(weights["wte"], dtype).T
 
 

@@ -48,6 +48,9 @@ def test_workspace_bytes_and_config_checks():
     ]
     for c in bad:
         assert B.gpt2_workspace_bytes(c, 1, 1) == 0
+    # flags: the tanh-GELU bit is accepted, any other bit rejected
+    assert B.gpt2_workspace_bytes(B.make_config(12, 12, 768, 50257, 1024, B.GPT2_BF16, B.GPT2_FLAG_GELU_TANH), 4, 1024) == n
+    assert B.gpt2_workspace_bytes(B.make_config(12, 12, 768, 50257, 1024, B.GPT2_BF16, 2), 4, 1024) == 0
 
 
 def test_create_rejects_bad_arguments_on_the_host():

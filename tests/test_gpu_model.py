@@ -69,6 +69,59 @@ def test_small_case_all_fp32_debug_mode(G):
     assert abs(loss - ref_loss) <= 1e-4
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_gelu_tanh_flag(G, dtype):
+    """GPT2_FLAG_GELU_TANH: the MLP uses the tanh form; parity with the oracle
+    run with gelu_tanh (and, in fp32, clearly closer to it than to the erf form)."""
+    W = synthetic.make_weights(SMALL)
+    ids = synthetic.make_ids(SMALL)
+    model = G.GPT2Model.from_workload(SMALL, W, dtype=dtype, flags=G.GPT2_FLAG_GELU_TANH)
+    d_ids = torch.from_numpy(ids).cuda()
+    d_tg = torch.from_numpy(synthetic.next_token_targets(ids)).cuda()
+    logits, loss = model.forward_loss(d_ids, d_tg)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    z = logits.cpu().numpy()
+    ref = O.forward(W, ids, SMALL.n_head, act=O.gelu_tanh)
+    ref_loss, _ = O.shifted_cross_entropy(ref, ids)
+    if dtype == "bf16":
+        assert _cmp.rel_l2(z, ref) <= _cmp.BF16_REL_L2
+        assert _cmp.max_abs(z, ref) <= _cmp.BF16_MAX_ABS
+        assert abs(float(loss.item()) - ref_loss) <= _cmp.BF16_LOSS_ABS
+    else:
+        assert _cmp.rel_l2(z, ref) <= _cmp.FP32_REL_L2
+        assert abs(float(loss.item()) - ref_loss) <= 1e-4
+        ref_erf = O.forward(W, ids, SMALL.n_head)
+        assert _cmp.rel_l2(z, ref) * 10 < _cmp.rel_l2(z, ref_erf)
+    model.close()
+
+
+def test_model_with_device_filled_sinusoidal_wpe(G):
+    """A model whose wpe is the fixed sinusoidal table filled on the device
+    (gpt2_fill_sinusoidal_wpe) against the oracle with the oracle's table."""
+    wl = SMALL
+    W = synthetic.make_weights(wl)
+    W["wpe"] = synthetic.round_to_bf16(O.sinusoidal_wpe(wl.n_ctx, wl.n_embd).astype(np.float32))
+    Wd = G.upload_weights(synthetic.make_weights(wl), "bf16")
+    wpe = torch.empty(wl.n_ctx, wl.n_embd, dtype=torch.bfloat16, device="cuda")
+    G.gpt2_fill_sinusoidal_wpe(G.GPT2_BF16, wpe, wl.n_ctx, wl.n_embd)
+    Wd["wpe"] = wpe
+    ids = synthetic.make_ids(wl)
+    model = G.GPT2Model.from_workload(wl, Wd)
+    d_ids = torch.from_numpy(ids).cuda()
+    d_tg = torch.from_numpy(synthetic.next_token_targets(ids)).cuda()
+    logits, loss = model.forward_loss(d_ids, d_tg)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    z = logits.cpu().numpy()
+    ref = O.forward(W, ids, wl.n_head)
+    ref_loss, _ = O.shifted_cross_entropy(ref, ids)
+    assert _cmp.rel_l2(z, ref) <= _cmp.BF16_REL_L2
+    assert _cmp.max_abs(z, ref) <= _cmp.BF16_MAX_ABS
+    assert abs(float(loss.item()) - ref_loss) <= _cmp.BF16_LOSS_ABS
+    model.close()
+
+
 def test_head_dim_32_bf16(G):
     wl = synthetic.random_case(32, n_layer=1, n_head=4, n_embd=128, vocab=777, n_ctx=160, batch=2, seq=150)
     W, ids, model, z, loss, tok = run_case(G, wl)

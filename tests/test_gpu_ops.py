@@ -96,7 +96,7 @@ LINEAR_SHAPES = [
 
 
 @pytest.mark.parametrize("bn", ["64", "128", "192", "256", ""])
-@pytest.mark.parametrize("epi", [0, 1, 2])
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
 @pytest.mark.parametrize("shape", LINEAR_SHAPES)
 def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
     if bn:
@@ -118,6 +118,8 @@ def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
         out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
         if epi == 1:
             ref = O.gelu(ref)
+        if epi == 3:
+            ref = O.gelu_tanh(ref)
     G.gpt2_op_linear(G.GPT2_BF16, epi, dev(A, "bf16"), dev(W, "bf16"), dev(bias, "bf16"), M, N, K, out, st)
     torch.cuda.synchronize()
     got = out.float().cpu().numpy()
@@ -151,7 +153,7 @@ def test_gelu_epilogue_within_one_bf16_ulp(G):
     assert np.abs(got - exact).max() <= 2.0 ** -8 * 8
 
 
-@pytest.mark.parametrize("epi", [0, 1, 2])
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
 def test_linear_fp32_simt(G, epi):
     M, N, K = 130, 200, 72
     rng = np.random.default_rng(40 + epi)
@@ -167,6 +169,8 @@ def test_linear_fp32_simt(G, epi):
         out = torch.empty(M, N, dtype=torch.float32, device="cuda")
         if epi == 1:
             ref = O.gelu(ref)
+        if epi == 3:
+            ref = O.gelu_tanh(ref)
     G.gpt2_op_linear(G.GPT2_FP32, epi, dev(A, "fp32"), dev(W, "fp32"), dev(bias, "fp32"), M, N, K, out)
     assert max_abs(out.cpu().numpy(), ref) <= 2e-5
 
@@ -269,3 +273,22 @@ def test_lmhead_ce_no_targets_sets_status(G):
     torch.cuda.synchronize()
     assert math.isnan(float(loss.item()))
     assert int(st.item()) & 4
+
+
+# ------------------------------------------------------ sinusoidal position table
+
+
+@pytest.mark.parametrize("n_ctx,C", [(1024, 768), (7, 10), (1, 2)])
+def test_fill_sinusoidal_wpe(G, n_ctx, C):
+    ref = O.sinusoidal_wpe(n_ctx, C)
+    f32 = torch.empty(n_ctx, C, dtype=torch.float32, device="cuda")
+    G.gpt2_fill_sinusoidal_wpe(G.GPT2_FP32, f32, n_ctx, C)
+    torch.cuda.synchronize()
+    assert max_abs(f32.cpu().numpy(), ref) <= 1e-7          # one fp32 rounding of values in [-1, 1]
+    b16 = torch.empty(n_ctx, C, dtype=torch.bfloat16, device="cuda")
+    G.gpt2_fill_sinusoidal_wpe(G.GPT2_BF16, b16, n_ctx, C)
+    torch.cuda.synchronize()
+    got = b16.float().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -9 * 1.0001)   # within half a bf16 ulp
+    with pytest.raises(G.GPT2Error):
+        G.gpt2_fill_sinusoidal_wpe(G.GPT2_FP32, f32, n_ctx, C + 1)   # odd C

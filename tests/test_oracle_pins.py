@@ -103,6 +103,38 @@ def test_gelu_matches_math_erf_and_torch():
     assert np.allclose(O.gelu(pre), 0.5 * C * (1 + math.erf(C / math.sqrt(2))), atol=0, rtol=1e-15)
 
 
+def test_gelu_tanh_matches_torch_and_its_identities():
+    xs = np.linspace(-8, 8, 161)
+    g = O.gelu_tanh(xs)
+    # library routine: torch's tanh-approximate GELU in fp64
+    ref = F.gelu(torch.from_numpy(xs), approximate="tanh").numpy()
+    assert np.abs(g - ref).max() <= 1e-14
+    # 0.5 x (1 + tanh u) is odd-symmetric around x/2: g(x) - g(-x) = x exactly
+    assert np.abs((g - O.gelu_tanh(-xs)) - xs).max() <= 1e-14
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+    # it approximates the exact form to within 5e-4 (and is not identical to it)
+    d = np.abs(g - O.gelu(xs))
+    assert d.max() <= 5e-4 and d.max() >= 1e-5
+
+
+def test_sinusoidal_wpe_closed_forms():
+    n_ctx, C = 64, 16
+    pe = O.sinusoidal_wpe(n_ctx, C)
+    assert pe.shape == (n_ctx, C)
+    # position 0: sin 0 = 0 in even columns, cos 0 = 1 in odd columns
+    assert np.array_equal(pe[0], np.tile([0.0, 1.0], C // 2))
+    # pair i = 0 has frequency 1: columns 0 and 1 are sin(pos), cos(pos)
+    pos = np.arange(n_ctx)
+    assert np.abs(pe[:, 0] - np.sin(pos)).max() <= 1e-15
+    assert np.abs(pe[:, 1] - np.cos(pos)).max() <= 1e-15
+    # every (sin, cos) pair lies on the unit circle
+    assert np.abs(pe[:, 0::2] ** 2 + pe[:, 1::2] ** 2 - 1.0).max() <= 1e-14
+    # the angle of pair i at position 1 is 10000^(-2i/C): a geometric progression
+    ang = np.arctan2(pe[1, 0::2], pe[1, 1::2])
+    assert np.allclose(ang[1:] / ang[:-1], 10000.0 ** (-2.0 / C), rtol=1e-12, atol=0)
+    assert abs(ang[0] - 1.0) <= 1e-15
+
+
 def test_cross_entropy_matches_torch():
     rng = np.random.default_rng(2)
     B, T, V = 3, 9, 41
@@ -357,3 +389,21 @@ def test_planted_dropped_attention_branch_is_caught(monkeypatch):
     orig_linear = O.linear
     monkeypatch.setattr(O, "linear", lambda x, w, b: orig_linear(x, w, b) if w.shape[0] != w.shape[1] else orig_linear(x, w, b) * 0)
     assert _fails(test_full_model_matches_torch_library_composition)
+
+
+def test_planted_sinusoidal_exponent_is_caught(monkeypatch):
+    def pe_wrong(n_ctx, C):   # i / C instead of 2i / C
+        pos = np.arange(n_ctx, dtype=np.float64)[:, None]
+        i = np.arange(C // 2, dtype=np.float64)[None, :]
+        a = pos / np.power(10000.0, i / C)
+        pe = np.empty((n_ctx, C))
+        pe[:, 0::2], pe[:, 1::2] = np.sin(a), np.cos(a)
+        return pe
+    monkeypatch.setattr(O, "sinusoidal_wpe", pe_wrong)
+    assert _fails(test_sinusoidal_wpe_closed_forms)
+
+
+def test_planted_gelu_tanh_coefficient_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "gelu_tanh",
+                        lambda x: 0.5 * x * (1 + np.tanh(math.sqrt(2 / math.pi) * (x + 0.0447 * x ** 3))))
+    assert _fails(test_gelu_tanh_matches_torch_and_its_identities)

@@ -8,6 +8,7 @@ handle. Importing this package fails if libgpt2.so has not been built.
 from . import binding  # noqa: F401  (raises ImportError when libgpt2.so is missing)
 from .binding import (  # noqa: F401
     GPT2_BF16, GPT2_FP32, GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID, GPT2Error,
+    GPT2_EPI_BIAS_GELU_TANH, GPT2_FLAG_GELU_TANH, gpt2_fill_sinusoidal_wpe,
     gpt2_workspace_bytes, gpt2_create, gpt2_forward, gpt2_loss, gpt2_forward_loss, gpt2_status,
     gpt2_error_string, gpt2_destroy, gpt2_launch_count, gpt2_set_timing_events, GPT2_TIMED_LMHEAD,
     gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear,

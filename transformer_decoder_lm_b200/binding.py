@@ -17,7 +17,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgpt2.so")
 
 GPT2_BF16, GPT2_FP32 = 0, 1
-GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID = 0, 1, 2
+GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID, GPT2_EPI_BIAS_GELU_TANH = 0, 1, 2, 3
+GPT2_FLAG_GELU_TANH = 1
 ERRORS = {
     0: "GPT2_OK", 1: "GPT2_ERR_INVALID_ARG", 2: "GPT2_ERR_UNSUPPORTED", 3: "GPT2_ERR_CUDA",
     4: "GPT2_ERR_WORKSPACE", 5: "GPT2_ERR_BAD_TOKEN", 6: "GPT2_ERR_DEVICE_TIMEOUT", 7: "GPT2_ERR_NO_TARGETS",
@@ -74,6 +75,7 @@ def _load():
         "gpt2_op_layernorm": (i, [i, vp, vp, vp, i, i, vp, vp]),
         "gpt2_op_linear": (i, [i, i, vp, vp, vp, i, i, i, vp, vp, vp]),
         "gpt2_op_attention": (i, [i, vp, i, i, i, i, vp, vp, vp]),
+        "gpt2_fill_sinusoidal_wpe": (i, [i, vp, i, i, vp]),
         "gpt2_op_lmhead_ce_workspace_bytes": (sz, [i, i, i]),
         "gpt2_op_lmhead_ce": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
         "gpt2_op_lmhead_ce_noalloc": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, vp]),
@@ -108,8 +110,9 @@ def _check(rc: int, where: str) -> None:
         raise GPT2Error(rc, where)
 
 
-def make_config(n_layer: int, n_head: int, n_embd: int, vocab: int, n_ctx: int, dtype: int) -> gpt2_config_t:
-    return gpt2_config_t(n_layer, n_head, n_embd, vocab, n_ctx, dtype, 0)
+def make_config(n_layer: int, n_head: int, n_embd: int, vocab: int, n_ctx: int, dtype: int,
+                flags: int = 0) -> gpt2_config_t:
+    return gpt2_config_t(n_layer, n_head, n_embd, vocab, n_ctx, dtype, flags)
 
 
 def gpt2_workspace_bytes(cfg: gpt2_config_t, max_B: int, max_T: int) -> int:
@@ -191,6 +194,10 @@ def gpt2_op_layernorm(dtype, x, g, b, M, C, out, stream=None):
 def gpt2_op_linear(dtype, epilogue, A, W, bias, M, N, K, out, status=None, stream=None):
     _check(lib.gpt2_op_linear(dtype, epilogue, _ptr(A), _ptr(W), _ptr(bias), M, N, K, _ptr(out), _ptr(status),
                               _stream(stream)), "gpt2_op_linear")
+
+
+def gpt2_fill_sinusoidal_wpe(dtype, wpe, n_ctx, C, stream=None):
+    _check(lib.gpt2_fill_sinusoidal_wpe(dtype, _ptr(wpe), n_ctx, C, _stream(stream)), "gpt2_fill_sinusoidal_wpe")
 
 
 def gpt2_op_attention(dtype, qkv, B, T, H, C, y, status=None, stream=None):

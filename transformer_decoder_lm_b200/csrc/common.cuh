@@ -387,6 +387,21 @@ __device__ __forceinline__ uint64_t gelu_erf_x2(uint64_t x) {
   return f2_fma(h, r, f2_pack(fmaxf(x0, 0.f), fmaxf(x1, 0.f)));
 }
 
+// Tanh-form GELU on a pair in packed fp32:
+//   0.5 x (1 + tanh u) = x / (1 + e^(-2u)),  u = sqrt(2/pi) (x + 0.044715 x^3),
+// with e^(-2u) = 2^(-2u log2 e) and the reciprocal on the SFU. Large |x|
+// saturates cleanly: e^(-2u) -> inf gives -0, -> 0 gives x.
+__device__ __forceinline__ uint64_t gelu_tanh_x2(uint64_t x) {
+  const uint64_t sq = f2_mul(x, x);
+  const uint64_t inner = f2_fma(f2_mul(sq, f2_pack(0.044715f, 0.044715f)), x, x);   // x + 0.044715 x^3
+  // -2 sqrt(2/pi) log2(e)
+  const uint64_t t = f2_mul(inner, f2_pack(-2.302208198144325f, -2.302208198144325f));
+  float t0, t1, x0, x1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(x, x0, x1);
+  return f2_pack(x0 * rcp_approx(1.f + ex2_approx(t0)), x1 * rcp_approx(1.f + ex2_approx(t1)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

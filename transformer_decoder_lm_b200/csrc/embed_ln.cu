@@ -182,4 +182,33 @@ cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const vo
   return cudaGetLastError();
 }
 
+// Fixed sinusoidal position table ("Hand-writing GPT-2 from scratch: the
+// Transformer decoder core modules in PyTorch", section 3.1): element
+// (pos, j) of [n_ctx, C] is sin (j even) or cos (j odd) of
+// pos / 10000^(2 (j / 2) / C), computed in double and rounded once.
+template <typename T>
+__global__ void sinusoidal_wpe_kernel(T* __restrict__ wpe, int n_ctx, int C) {
+  const long long n = (long long)n_ctx * C;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int pos = (int)(idx / C), j = (int)(idx % C), i = j >> 1;
+    const double angle = (double)pos / pow(10000.0, (2.0 * i) / C);
+    const double v = (j & 1) ? cos(angle) : sin(angle);
+    if constexpr (sizeof(T) == 2)
+      wpe[idx] = __double2bfloat16(v);
+    else
+      wpe[idx] = (float)v;
+  }
+}
+
+cudaError_t sinusoidal_wpe_launch(bool bf16_, void* wpe, int n_ctx, int C, cudaStream_t s) {
+  const long long n = (long long)n_ctx * C;
+  const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  if (bf16_)
+    sinusoidal_wpe_kernel<bf16><<<grid, 256, 0, s>>>(static_cast<bf16*>(wpe), n_ctx, C);
+  else
+    sinusoidal_wpe_kernel<float><<<grid, 256, 0, s>>>(static_cast<float*>(wpe), n_ctx, C);
+  return cudaGetLastError();
+}
+
 }  // namespace g2

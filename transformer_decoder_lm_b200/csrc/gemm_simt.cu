@@ -67,7 +67,9 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const float* __restrict_
       v += bias[n];
       float* o = static_cast<float*>(args.out) + (size_t)m * args.ldo + n;
       if (EPI == EPI_BIAS) *o = v;
-      if (EPI == EPI_GELU) *o = 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+      if (EPI == EPI_GELU)
+        *o = args.gelu_tanh ? 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)))
+                            : 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
       if (EPI == EPI_RESID) *o += v;
     }
   }

@@ -386,7 +386,8 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
               const float b0 = __uint_as_float(bc[j] << 16), b1 = __uint_as_float(bc[j] & 0xffff0000u);
               const float x0 = __uint_as_float(v[c][2 * j]), x1 = __uint_as_float(v[c][2 * j + 1]);
               if (EPI == EPI_GELU) {
-                const uint64_t y2 = gelu_erf_x2(f2_add(f2_pack(x0, x1), f2_pack(b0, b1)));
+                const uint64_t z2 = f2_add(f2_pack(x0, x1), f2_pack(b0, b1));
+                const uint64_t y2 = args.gelu_tanh ? gelu_tanh_x2(z2) : gelu_erf_x2(z2);
                 float a, b;
                 f2_unpack(y2, a, b);
                 pk[j] = pack_bf16x2(a, b);

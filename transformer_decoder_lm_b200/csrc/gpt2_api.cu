@@ -81,7 +81,7 @@ int check_config(const gpt2_config_t* c) {
   if (!c) return GPT2_ERR_INVALID_ARG;
   if (c->n_layer < 1 || c->n_head < 1 || c->n_embd < 1 || c->vocab < 1 || c->n_ctx < 1) return GPT2_ERR_INVALID_ARG;
   if (c->dtype != GPT2_BF16 && c->dtype != GPT2_FP32) return GPT2_ERR_INVALID_ARG;
-  if (c->flags != 0) return GPT2_ERR_INVALID_ARG;
+  if (c->flags & ~GPT2_FLAG_GELU_TANH) return GPT2_ERR_INVALID_ARG;
   if (c->n_embd % c->n_head) return GPT2_ERR_UNSUPPORTED;
   const int D = c->n_embd / c->n_head;
   if (D != 32 && D != 64) return GPT2_ERR_UNSUPPORTED;
@@ -155,6 +155,7 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   a.out = out;
   a.ldo = ldo;
   a.status = m->status;
+  a.gelu_tanh = (m->cfg.flags & GPT2_FLAG_GELU_TANH) ? 1 : 0;
   cudaError_t e;
   if (m->bf16) {
     const int bn = gemm_tc_pick_bn(M, N, m->num_sms, epi);
@@ -440,7 +441,7 @@ int gpt2_op_layernorm(int dtype, const float* x, const void* g, const void* b, i
 
 int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const void* bias, int M, int N, int K,
                    void* out, int* status, void* stream) {
-  if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || epilogue < 0 || epilogue > 2 || !aligned16(A) || !aligned16(W) ||
+  if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || epilogue < 0 || epilogue > 3 || !aligned16(A) || !aligned16(W) ||
       !aligned16(bias) || !aligned16(out) || M < 0 || N < 8 || K < 8 || (N % 8) || (K % 8))
     return GPT2_ERR_INVALID_ARG;
   if (M == 0) return GPT2_OK;
@@ -453,6 +454,10 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
   a.out = out;
   a.ldo = N;
   a.status = status;
+  if (epilogue == GPT2_EPI_BIAS_GELU_TANH) {   // the GELU epilogue with the tanh form
+    epilogue = EPI_GELU;
+    a.gelu_tanh = 1;
+  }
   if (dtype == GPT2_FP32)
     return gemm_simt_launch(epilogue, static_cast<const float*>(A), static_cast<const float*>(W), a, s) == cudaSuccess
                ? GPT2_OK
@@ -468,6 +473,13 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
                                                      : make_tmap_out_bf16(&tc, out, M, N, N);
   if (!ok_c) return GPT2_ERR_CUDA;
   return gemm_tc_launch(epilogue, bn, ta, tb, tc, a, sms, s) == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+}
+
+int gpt2_fill_sinusoidal_wpe(int dtype, void* wpe, int n_ctx, int C, void* stream) {
+  if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || !wpe || n_ctx < 1 || C < 2 || (C % 2)) return GPT2_ERR_INVALID_ARG;
+  return sinusoidal_wpe_launch(dtype == GPT2_BF16, wpe, n_ctx, C, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? GPT2_OK
+             : GPT2_ERR_CUDA;
 }
 
 int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, void* y, int* status, void* stream) {

@@ -41,6 +41,7 @@ struct GemmArgs {
   float2* part;            // EPI_LMHEAD: per (column group, row) (max, sum exp(z - max)), [n_groups, M]
   float* tgt_logit;        // EPI_LMHEAD: [M] logit of the target column
   int* status;
+  int gelu_tanh;           // EPI_GELU: 1 = tanh approximation, 0 = exact erf form
 };
 
 // ---- tensor maps (host) -------------------------------------------------
@@ -83,6 +84,9 @@ cudaError_t embed_launch(bool bf16, const int* ids, const void* wte, const void*
                          int C, int V, int* status, cudaStream_t s);
 cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const void* b, void* out, int M, int C,
                              cudaStream_t s);
+
+// ---- sinusoidal position table (bf16 or fp32 [n_ctx, C]) -------------------
+cudaError_t sinusoidal_wpe_launch(bool bf16, void* wpe, int n_ctx, int C, cudaStream_t s);
 
 // ---- attention ---------------------------------------------------------------
 // tcgen05 flash attention (bf16, d_head 64); attention_launch dispatches to it.

@@ -37,10 +37,11 @@ class GPT2Model:
     max_B, max_T: the largest batch the workspace is sized for.
     """
 
-    def __init__(self, n_layer, n_head, n_embd, vocab, n_ctx, dtype, weights, max_B, max_T, device="cuda"):
+    def __init__(self, n_layer, n_head, n_embd, vocab, n_ctx, dtype, weights, max_B, max_T, device="cuda",
+                 flags=0):
         self.dtype = dtype
         self.cfg = B.make_config(n_layer, n_head, n_embd, vocab, n_ctx,
-                                 B.GPT2_BF16 if dtype == "bf16" else B.GPT2_FP32)
+                                 B.GPT2_BF16 if dtype == "bf16" else B.GPT2_FP32, flags)
         if isinstance(weights["wte"], np.ndarray):
             weights = upload_weights(weights, dtype, device)
         self.weights = weights
@@ -52,9 +53,9 @@ class GPT2Model:
         self.handle, self._keep = B.gpt2_create(self.cfg, weights, self.workspace, max_B, max_T)
 
     @classmethod
-    def from_workload(cls, wl, weights, max_B=None, max_T=None, dtype=None, device="cuda"):
+    def from_workload(cls, wl, weights, max_B=None, max_T=None, dtype=None, device="cuda", flags=0):
         return cls(wl.n_layer, wl.n_head, wl.n_embd, wl.vocab, wl.n_ctx, dtype or wl.dtype, weights,
-                   max_B or wl.batch, max_T or wl.seq, device)
+                   max_B or wl.batch, max_T or wl.seq, device, flags)
 
     def forward(self, ids: torch.Tensor, logits: Optional[torch.Tensor] = None, want_logits=True, stream=None):
         Bsz, T = ids.shape
