@@ -397,6 +397,21 @@ def run_kernel(args):
         out = torch.empty(M, C, dtype=bf, device="cuda")
         fn = lambda: G.gpt2_op_layernorm(G.GPT2_BF16, x, g, b, M, C, out)
         flops = 0.0
+    elif k == "decode":
+        # one incremental decoding step of the 124M model for 4 sequences at
+        # position 1023 (context 1024), after a prefill of positions 0..1022
+        model = G.GPT2Model.from_workload(WL, synthetic.make_weights(WL))
+        cache = model.new_kv_cache()
+        ids = torch.from_numpy(synthetic.make_ids(WL)).cuda()
+        pos = WL.seq - 1
+        model.prefill(ids[:, :pos].contiguous(), cache, want_logits=False)
+        new = ids[:, pos].contiguous()
+        dlog = torch.empty(WL.batch, V, dtype=torch.float32, device="cuda")
+        fn = lambda: model.decode_step(new, pos, cache, logits=dlog)
+        flops = 0.0
+        es = 2
+        n_block = WL.n_layer * (12 * C * C + 13 * C)   # Linear weights + biases + LN of the blocks
+        decode_bytes = es * (n_block + V * C) + es * WL.n_layer * WL.batch * WL.seq * 2 * C
     else:
         raise SystemExit(f"unknown kernel {k}")
     for _ in range(args.warmup):
@@ -424,15 +439,21 @@ def run_kernel(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / (reps * per_graph)
-    print(json.dumps({"kernel": k, "ms_per_launch": ms, "tflops": flops / (ms / 1e3) / 1e12 if flops else None,
-                      "launches": reps * per_graph, "timing": "CUDA graph replay"}), flush=True)
+    line = {"kernel": k, "ms_per_launch": ms, "tflops": flops / (ms / 1e3) / 1e12 if flops else None,
+            "launches": reps * per_graph, "timing": "CUDA graph replay"}
+    if k == "decode":
+        hbm = peaks()[0]
+        line.update({"tokens_per_s": WL.batch / (ms / 1e3), "context": WL.seq,
+                     "min_bytes_per_step": decode_bytes, "gbs": decode_bytes / (ms / 1e3) / 1e9,
+                     "hbm_frac": decode_bytes / (ms / 1e3) / 1e9 / hbm})
+    print(json.dumps(line), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None,
                     help="run one step alone: lmhead, lmhead_ce (no logits), c_attn, attn_proj, c_fc, mlp_proj, "
-                         "attention, layernorm")
+                         "attention, layernorm, decode (one key/value-cache decoding step, B 4, context 1024)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)

@@ -196,6 +196,36 @@ enum { GPT2_EPI_BIAS = 0, GPT2_EPI_BIAS_GELU = 1, GPT2_EPI_BIAS_RESID = 2, GPT2_
 int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const void* bias,
                    int M, int N, int K, void* out, int* status, void* stream);
 
+/* ---- incremental decoding with a key/value cache ---------------------------
+ * The pages' generate loops feed the sequence back one new token at a time
+ * and keep every layer's keys and values of the earlier positions
+ * ("Hand-writing GPT-2 from scratch: the Transformer decoder core modules in
+ * PyTorch", section 6.3, past_key_values; "GPT-2 model development in
+ * practice: from principles to deployment", section 4.1). With the cache, a
+ * new position costs one row through every Linear and one query against the
+ * cached keys, and its logits equal row `pos` of the full forward over
+ * positions 0..pos.
+ *
+ * Cache layout, `dtype` elements: [n_layer][max_B][n_ctx][2C], position t of
+ * sequence b of layer l holding k (C values, heads concatenated) then v (C
+ * values). max_B is the one given to gpt2_create; the caller allocates the
+ * cache (gpt2_kv_cache_bytes, 0 for a bad config) and owns it. */
+size_t gpt2_kv_cache_bytes(const gpt2_config_t* cfg, int max_B);
+
+/* The forward pass of gpt2_forward over ids [B, T] that also stores every
+ * layer's k and v of positions 0..T-1 of each sequence in the cache.
+ * logits_or_null as in gpt2_forward. */
+int gpt2_prefill(gpt2_handle_t h, void* kv_cache, const int32_t* ids, int B, int T,
+                 float* logits_or_null, void* stream);
+
+/* One new token per sequence at position pos (0 <= pos < n_ctx): ids_new
+ * int32 [B]; the cache must hold positions 0..pos-1 of these B sequences
+ * (from gpt2_prefill or earlier steps). Stores the new position's k and v in
+ * the cache and writes logits fp32 [B, vocab] of the new position.
+ * GPT2_ERR_UNSUPPORTED if pos >= n_ctx; GPT2_ERR_INVALID_ARG if B > max_B. */
+int gpt2_decode_step(gpt2_handle_t h, void* kv_cache, const int32_t* ids_new, int B, int pos,
+                     float* logits, void* stream);
+
 /* Fixed sinusoidal position table ("Hand-writing GPT-2 from scratch: the
  * Transformer decoder core modules in PyTorch", section 3.1, a variant the
  * other pages do not use: they learn wpe): for pos in [0, n_ctx) and i in

@@ -9,6 +9,7 @@ from . import binding  # noqa: F401  (raises ImportError when libgpt2.so is miss
 from .binding import (  # noqa: F401
     GPT2_BF16, GPT2_FP32, GPT2_EPI_BIAS, GPT2_EPI_BIAS_GELU, GPT2_EPI_BIAS_RESID, GPT2Error,
     GPT2_EPI_BIAS_GELU_TANH, GPT2_FLAG_GELU_TANH, gpt2_fill_sinusoidal_wpe,
+    gpt2_kv_cache_bytes, gpt2_prefill, gpt2_decode_step,
     gpt2_workspace_bytes, gpt2_create, gpt2_forward, gpt2_loss, gpt2_forward_loss, gpt2_status,
     gpt2_error_string, gpt2_destroy, gpt2_launch_count, gpt2_set_timing_events, GPT2_TIMED_LMHEAD,
     gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear,

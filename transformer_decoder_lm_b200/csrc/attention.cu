@@ -277,4 +277,96 @@ cudaError_t attention_launch(bool bf16_, const void* qkv, void* y, int B, int T,
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- decode
+// One new query per (sequence b, head h) against the cached keys and values
+// of positions 0..len-1 (the new one included): the scores go to shared
+// memory, then max, exp and sum, then every thread (d = tid % D) sums
+// p_j v_j[d] over one residue class of j; the classes are added in a fixed
+// order (deterministic). Memory-bound: each cached row is read once.
+template <typename T>
+__device__ __forceinline__ float dec_to_f(T v);
+template <>
+__device__ __forceinline__ float dec_to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float dec_to_f<bf16>(bf16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__global__ void __launch_bounds__(128) attn_decode_kernel(const T* __restrict__ qkv, const T* __restrict__ cache,
+                                                          T* __restrict__ y, int C, int n_ctx, int len, float scale) {
+  extern __shared__ float dsm[];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int D = C / gridDim.x;
+  float* q = dsm;              // [D]
+  float* p = dsm + D;          // [len]
+  float* red = p + len;        // [128]
+  const T* qrow = qkv + (size_t)b * 3 * C + h * D;
+  for (int d = tid; d < D; d += 128) q[d] = dec_to_f(qrow[d]);
+  __syncthreads();
+  const T* kb = cache + (size_t)b * n_ctx * 2 * C + h * D;   // row t at kb + t * 2C
+  const T* vb = kb + C;
+  float mx = -INFINITY;
+  for (int j = tid; j < len; j += 128) {
+    const T* kr = kb + (size_t)j * 2 * C;
+    float sc = 0.f;
+    for (int d = 0; d < D; ++d) sc = fmaf(q[d], dec_to_f(kr[d]), sc);
+    sc *= scale;
+    p[j] = sc;
+    mx = fmaxf(mx, sc);
+  }
+  red[tid] = mx;
+  __syncthreads();
+  for (int o = 64; o > 0; o >>= 1) {
+    if (tid < o) red[tid] = fmaxf(red[tid], red[tid + o]);
+    __syncthreads();
+  }
+  mx = red[0];
+  __syncthreads();
+  float sum = 0.f;
+  for (int j = tid; j < len; j += 128) {
+    const float e = expf(p[j] - mx);
+    p[j] = e;
+    sum += e;
+  }
+  red[tid] = sum;
+  __syncthreads();
+  for (int o = 64; o > 0; o >>= 1) {
+    if (tid < o) red[tid] += red[tid + o];
+    __syncthreads();
+  }
+  sum = red[0];
+  __syncthreads();
+  const int G = 128 / D, d = tid % D, g = tid / D;
+  float acc = 0.f;
+  for (int j = g; j < len; j += G) acc = fmaf(p[j], dec_to_f(vb[(size_t)j * 2 * C + d]), acc);
+  red[tid] = acc;
+  __syncthreads();
+  if (g == 0) {
+    for (int k = 1; k < G; ++k) acc += red[k * D + d];
+    const float out = acc / sum;
+    if constexpr (sizeof(T) == 2)
+      y[(size_t)b * C + h * D + d] = __float2bfloat16_rn(out);
+    else
+      y[(size_t)b * C + h * D + d] = out;
+  }
+}
+
+cudaError_t attention_decode_launch(bool bf16_, const void* qkv, const void* cache, void* y, int B, int H, int C,
+                                    int n_ctx, int len, cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  const int D = C / H;
+  if (D < 1 || D > 128 || 128 % D || len < 1 || len > n_ctx) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)(D + len + 128) * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  const float scale = (float)(1.0 / sqrt((double)D));
+  dim3 grid(H, B);
+  if (bf16_)
+    attn_decode_kernel<bf16><<<grid, 128, smem, s>>>(static_cast<const bf16*>(qkv), static_cast<const bf16*>(cache),
+                                                     static_cast<bf16*>(y), C, n_ctx, len, scale);
+  else
+    attn_decode_kernel<float><<<grid, 128, smem, s>>>(static_cast<const float*>(qkv),
+                                                      static_cast<const float*>(cache), static_cast<float*>(y), C,
+                                                      n_ctx, len, scale);
+  return cudaGetLastError();
+}
+
 }  // namespace g2

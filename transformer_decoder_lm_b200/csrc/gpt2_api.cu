@@ -166,8 +166,14 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
+// Bytes of one layer's slice of a key/value cache: [max_B][n_ctx][2C].
+size_t kv_layer_bytes(const gpt2_model* m) {
+  const size_t es = m->bf16 ? 2 : 4;
+  return (size_t)m->max_B * m->cfg.n_ctx * 2 * m->cfg.n_embd * es;
+}
+
 int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B, int T, float* logits,
-                float* loss_out, float* tok_out, cudaStream_t s) {
+                float* loss_out, float* tok_out, cudaStream_t s, void* kv_cache = nullptr) {
   if (!m || !ids || B < 1 || T < 1) return GPT2_ERR_INVALID_ARG;
   if (B > m->max_B || T > m->max_T) return GPT2_ERR_INVALID_ARG;
   if (T > m->cfg.n_ctx) return GPT2_ERR_UNSUPPORTED;
@@ -203,6 +209,14 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
     G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C, m->qkv, 3 * C, s));
+    if (kv_cache) {   // k and v of positions 0..T-1 of every sequence into this layer's cache
+      const size_t es = m->bf16 ? 2 : 4;
+      uint8_t* cl = static_cast<uint8_t*>(kv_cache) + (size_t)l * kv_layer_bytes(m);
+      for (int b = 0; b < B; ++b)
+        G2_CK(cudaMemcpy2DAsync(cl + (size_t)b * c.n_ctx * 2 * C * es, 2 * C * es,
+                                static_cast<uint8_t*>(m->qkv) + ((size_t)b * T * 3 * C + C) * es, 3 * C * es,
+                                2 * C * es, T, cudaMemcpyDeviceToDevice, s));
+    }
     G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, &m->attn, m->status, s));
     G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
@@ -243,6 +257,82 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
       m->launches += loss_out ? 2 : 1;
     }
   }
+#undef G2_CK
+#undef G2_RC
+  return rc;
+}
+
+// One new token per sequence at position pos, against the key/value cache
+// (gpt2_decode_step): every row-wise step of run_forward on B rows, the new
+// k and v stored at `pos`, attention of the one query over positions 0..pos.
+int run_decode(gpt2_model* m, void* kv_cache, const int32_t* ids, int B, int pos, float* logits, cudaStream_t s) {
+  if (!m || !kv_cache || !ids || !logits || B < 1 || B > m->max_B || pos < 0) return GPT2_ERR_INVALID_ARG;
+  if (pos >= m->cfg.n_ctx) return GPT2_ERR_UNSUPPORTED;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return GPT2_ERR_CUDA;
+  if (cur != m->device && cudaSetDevice(m->device) != cudaSuccess) return GPT2_ERR_CUDA;
+  const gpt2_config_t& c = m->cfg;
+  const int M = B, C = c.n_embd, H = c.n_head, V = c.vocab;
+  const size_t es = m->bf16 ? 2 : 4;
+  CUtensorMap tm_h, tm_y, tm_f, out_qkv, out_f, out_x;
+  if (m->bf16) {
+    if (!make_tmap_bf16(&tm_h, m->h, M, C, C, 128) || !make_tmap_bf16(&tm_y, m->y, M, C, C, 128) ||
+        !make_tmap_bf16(&tm_f, m->f, M, 4 * C, 4 * C, 128) ||
+        !make_tmap_out_bf16(&out_qkv, m->qkv, M, 3 * C, 3 * C) || !make_tmap_out_bf16(&out_f, m->f, M, 4 * C, 4 * C) ||
+        !make_tmap_out_f32(&out_x, m->x, M, C, C))
+      return GPT2_ERR_CUDA;
+  }
+  int rc = GPT2_OK;
+#define G2_CK(expr)                                  \
+  do {                                               \
+    if ((expr) != cudaSuccess) return GPT2_ERR_CUDA; \
+  } while (0)
+#define G2_RC(expr)                  \
+  do {                               \
+    rc = (expr);                     \
+    if (rc != GPT2_OK) return rc;    \
+  } while (0)
+  // x = wte[id] + wpe[pos]: the embedding of one position per row
+  const void* wpe_pos = static_cast<const uint8_t*>(m->wpe) + (size_t)pos * C * es;
+  G2_CK(embed_launch(m->bf16, ids, m->wte, wpe_pos, m->x, M, 1, C, V, m->status, s));
+  for (int l = 0; l < c.n_layer; ++l) {
+    const LayerPtrs& L = m->layers[l];
+    const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
+    uint8_t* cl = static_cast<uint8_t*>(kv_cache) + (size_t)l * kv_layer_bytes(m);
+    G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
+    G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C,
+                     m->qkv, 3 * C, s));
+    // the new k and v at position pos of each sequence
+    G2_CK(cudaMemcpy2DAsync(cl + (size_t)pos * 2 * C * es, (size_t)c.n_ctx * 2 * C * es,
+                            static_cast<uint8_t*>(m->qkv) + (size_t)C * es, 3 * C * es, 2 * C * es, B,
+                            cudaMemcpyDeviceToDevice, s));
+    G2_CK(attention_decode_launch(m->bf16, m->qkv, cl, m->y, B, H, C, c.n_ctx, pos + 1, s));
+    G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C,
+                     m->x, C, s));
+    G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
+    G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, &out_f, L.fc_b, M, 4 * C, C, m->f, 4 * C,
+                     s));
+    G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, &out_x, L.mlp_proj_b, M, C,
+                     4 * C, m->x, C, s));
+    m->launches += 7;
+  }
+  G2_CK(layernorm_launch(m->bf16, m->x, m->lnf_g, m->lnf_b, m->h, M, C, s));
+  GemmArgs a{};
+  a.M = M;
+  a.N = V;
+  a.K = C;
+  a.out = logits;
+  a.ldo = V;
+  a.part = m->part;
+  a.tgt_logit = m->tgt;
+  a.status = m->status;
+  if (m->bf16) {
+    const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
+    G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, tm_h, m->wte_map[bn_index(bn)], tm_h, a, m->num_sms, s));
+  } else {
+    G2_CK(gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(m->h), static_cast<const float*>(m->wte), a, s));
+  }
+  m->launches += 3;
 #undef G2_CK
 #undef G2_RC
   return rc;
@@ -375,6 +465,25 @@ int gpt2_forward_loss(gpt2_handle_t h, const int32_t* ids, const int32_t* target
   if (!targets || !loss_out) return GPT2_ERR_INVALID_ARG;
   return run_forward(h, ids, targets, B, T, logits_or_null, loss_out, token_loss_or_null,
                      static_cast<cudaStream_t>(stream));
+}
+
+size_t gpt2_kv_cache_bytes(const gpt2_config_t* cfg, int max_B) {
+  if (check_config(cfg) != GPT2_OK || max_B < 1) return 0;
+  const size_t es = cfg->dtype == GPT2_BF16 ? 2 : 4;
+  return (size_t)cfg->n_layer * max_B * cfg->n_ctx * 2 * cfg->n_embd * es;
+}
+
+int gpt2_prefill(gpt2_handle_t h, void* kv_cache, const int32_t* ids, int B, int T, float* logits_or_null,
+                 void* stream) {
+  if (!kv_cache || !aligned16(kv_cache)) return GPT2_ERR_INVALID_ARG;
+  return run_forward(h, ids, nullptr, B, T, logits_or_null, nullptr, nullptr, static_cast<cudaStream_t>(stream),
+                     kv_cache);
+}
+
+int gpt2_decode_step(gpt2_handle_t h, void* kv_cache, const int32_t* ids_new, int B, int pos, float* logits,
+                     void* stream) {
+  if (!kv_cache || !aligned16(kv_cache)) return GPT2_ERR_INVALID_ARG;
+  return run_decode(h, kv_cache, ids_new, B, pos, logits, static_cast<cudaStream_t>(stream));
 }
 
 int gpt2_status(gpt2_handle_t h, void* stream) {

@@ -116,6 +116,13 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
 cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C,
                              const AttnScratch* scratch, int* status, cudaStream_t s);
 
+// One query per (sequence, head) against `len` cached positions: y [B, C] =
+// softmax(q k^T / sqrt(D)) v with q from qkv [B, 3C] and k, v from one
+// layer's cache [max_B][n_ctx][2C] (k then v per position). D = C / H must
+// divide 128.
+cudaError_t attention_decode_launch(bool bf16, const void* qkv, const void* cache, void* y, int B, int H, int C,
+                                    int n_ctx, int len, cudaStream_t s);
+
 // ---- cross-entropy finalisation -------------------------------------------
 // token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
 // target is negative); loss_out (if not NULL) = mean over scored rows.

@@ -50,6 +50,7 @@ class GPT2Model:
         if nbytes == 0:
             raise B.GPT2Error(B.ERR_CODE["GPT2_ERR_INVALID_ARG"], "gpt2_workspace_bytes")
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.max_B = max_B
         self.handle, self._keep = B.gpt2_create(self.cfg, weights, self.workspace, max_B, max_T)
 
     @classmethod
@@ -79,6 +80,26 @@ class GPT2Model:
             loss_out = torch.empty(1, dtype=torch.float32, device=ids.device)
         B.gpt2_forward_loss(self.handle, ids, targets, Bsz, T, logits, loss_out, token_loss, stream)
         return logits, loss_out
+
+    def new_kv_cache(self) -> torch.Tensor:
+        """A key/value cache for incremental decoding (gpt2_kv_cache_bytes bytes)."""
+        n = B.gpt2_kv_cache_bytes(self.cfg, self.max_B)
+        return torch.empty(n, dtype=torch.uint8, device=self.workspace.device)
+
+    def prefill(self, ids: torch.Tensor, kv_cache: torch.Tensor, want_logits=True, stream=None):
+        """The forward over ids [B, T], storing every layer's keys and values in kv_cache."""
+        Bsz, T = ids.shape
+        logits = torch.empty(Bsz, T, self.vocab, dtype=torch.float32, device=ids.device) if want_logits else None
+        B.gpt2_prefill(self.handle, kv_cache, ids, Bsz, T, logits, stream)
+        return logits
+
+    def decode_step(self, ids_new: torch.Tensor, pos: int, kv_cache: torch.Tensor, logits=None, stream=None):
+        """Logits [B, vocab] of one new token per sequence at position pos."""
+        Bsz = ids_new.shape[0]
+        if logits is None:
+            logits = torch.empty(Bsz, self.vocab, dtype=torch.float32, device=ids_new.device)
+        B.gpt2_decode_step(self.handle, kv_cache, ids_new, Bsz, pos, logits, stream)
+        return logits
 
     def status(self, stream=None) -> int:
         return B.gpt2_status(self.handle, stream)
