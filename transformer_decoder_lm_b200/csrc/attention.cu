@@ -350,14 +350,126 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const T* __restrict__ 
   }
 }
 
+// bf16 decode, split over the keys: block (h, b, split) takes up to 256
+// cached positions, one per thread for the scores (each key row read with
+// 16-byte loads), then (D/8 column groups) x (256 / (D/8) key classes) for
+// p v with 16-byte loads; it leaves (max, sum, unnormalised o[D]) in `part`.
+// attn_decode_combine_kernel merges the splits in a fixed order.
+constexpr int DEC_KEYS = 256;
+
+template <int D>
+__global__ void __launch_bounds__(DEC_KEYS) attn_decode_part_kernel(const bf16* __restrict__ qkv,
+                                                                    const bf16* __restrict__ cache,
+                                                                    float* __restrict__ part, int C, int n_ctx,
+                                                                    int len, float scale) {
+  constexpr int DG = D / 8, KG = DEC_KEYS / DG;
+  __shared__ float qs[D];
+  __shared__ float ps[DEC_KEYS];
+  __shared__ float red[DEC_KEYS / 32];
+  __shared__ float accs[KG][D];
+  const int h = blockIdx.x, b = blockIdx.y, sp = blockIdx.z, H = gridDim.x, S = gridDim.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j0 = sp * DEC_KEYS, n = min(len - j0, DEC_KEYS);   // n >= 1
+  if (tid < D) qs[tid] = __bfloat162float(qkv[(size_t)b * 3 * C + h * D + tid]);
+  __syncthreads();
+  const bf16* base = cache + (size_t)b * n_ctx * 2 * C + h * D;   // key row t at base + t * 2C, value at + C
+  float sc = -INFINITY;
+  if (tid < n) {
+    const uint4* kr = reinterpret_cast<const uint4*>(base + (size_t)(j0 + tid) * 2 * C);
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < DG; ++u) {
+      const uint4 w = kr[u];
+      const bf16* e = reinterpret_cast<const bf16*>(&w);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc = fmaf(qs[u * 8 + k], __bfloat162float(e[k]), acc);
+    }
+    sc = acc * scale;
+  }
+  float mx = sc;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int w = 1; w < DEC_KEYS / 32; ++w) mx = fmaxf(mx, red[w]);
+  __syncthreads();
+  const float e = tid < n ? expf(sc - mx) : 0.f;
+  ps[tid] = e;
+  float sum = e;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  sum = 0.f;
+#pragma unroll
+  for (int w = 0; w < DEC_KEYS / 32; ++w) sum += red[w];
+  const int dg = tid % DG, kg = tid / DG;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int jj = kg; jj < n; jj += KG) {
+    const uint4 w = *reinterpret_cast<const uint4*>(base + (size_t)(j0 + jj) * 2 * C + C + dg * 8);
+    const bf16* v = reinterpret_cast<const bf16*>(&w);
+    const float pj = ps[jj];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(pj, __bfloat162float(v[k]), acc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) accs[kg][dg * 8 + k] = acc[k];
+  __syncthreads();
+  float* pp = part + ((size_t)(b * H + h) * S + sp) * (D + 2);
+  if (tid < D) {
+    float o = 0.f;
+    for (int k = 0; k < KG; ++k) o += accs[k][tid];
+    pp[2 + tid] = o;
+  }
+  if (tid == 0) {
+    pp[0] = mx;
+    pp[1] = sum;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) attn_decode_combine_kernel(const float* __restrict__ part, bf16* __restrict__ y,
+                                                                int C, int S) {
+  const int h = blockIdx.x, b = blockIdx.y, H = gridDim.x, d = threadIdx.x;
+  const float* pp = part + (size_t)(b * H + h) * S * (D + 2);
+  float m = -INFINITY;
+  for (int s = 0; s < S; ++s) m = fmaxf(m, pp[s * (D + 2)]);
+  float l = 0.f, o = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float f = expf(pp[s * (D + 2)] - m);
+    l = fmaf(pp[s * (D + 2) + 1], f, l);
+    o = fmaf(pp[s * (D + 2) + 2 + d], f, o);
+  }
+  y[(size_t)b * C + h * D + d] = __float2bfloat16_rn(o / l);
+}
+
+template <int D>
+cudaError_t decode_split_launch(const void* qkv, const void* cache, void* y, float* part, int B, int H, int C,
+                                int n_ctx, int len, float scale, cudaStream_t s) {
+  const int S = (len + DEC_KEYS - 1) / DEC_KEYS;
+  attn_decode_part_kernel<D><<<dim3(H, B, S), DEC_KEYS, 0, s>>>(static_cast<const bf16*>(qkv),
+                                                                static_cast<const bf16*>(cache), part, C, n_ctx, len,
+                                                                scale);
+  attn_decode_combine_kernel<D><<<dim3(H, B), D, 0, s>>>(part, static_cast<bf16*>(y), C, S);
+  return cudaGetLastError();
+}
+
 cudaError_t attention_decode_launch(bool bf16_, const void* qkv, const void* cache, void* y, int B, int H, int C,
-                                    int n_ctx, int len, cudaStream_t s) {
+                                    int n_ctx, int len, float* part, size_t part_floats, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
   const int D = C / H;
   if (D < 1 || D > 128 || 128 % D || len < 1 || len > n_ctx) return cudaErrorInvalidValue;
+  const float scale = (float)(1.0 / sqrt((double)D));
+  const int S = (len + DEC_KEYS - 1) / DEC_KEYS;
+  const bool split_ok = part != nullptr && (size_t)B * H * S * (D + 2) <= part_floats;
+  if (bf16_ && split_ok && (D == 64 || D == 32)) {
+    if (D == 64) return decode_split_launch<64>(qkv, cache, y, part, B, H, C, n_ctx, len, scale, s);
+    return decode_split_launch<32>(qkv, cache, y, part, B, H, C, n_ctx, len, scale, s);
+  }
   const size_t smem = (size_t)(D + len + 128) * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  const float scale = (float)(1.0 / sqrt((double)D));
   dim3 grid(H, B);
   if (bf16_)
     attn_decode_kernel<bf16><<<grid, 128, smem, s>>>(static_cast<const bf16*>(qkv), static_cast<const bf16*>(cache),

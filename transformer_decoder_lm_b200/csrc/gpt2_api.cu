@@ -306,7 +306,9 @@ int run_decode(gpt2_model* m, void* kv_cache, const int32_t* ids, int B, int pos
     G2_CK(cudaMemcpy2DAsync(cl + (size_t)pos * 2 * C * es, (size_t)c.n_ctx * 2 * C * es,
                             static_cast<uint8_t*>(m->qkv) + (size_t)C * es, 3 * C * es, 2 * C * es, B,
                             cudaMemcpyDeviceToDevice, s));
-    G2_CK(attention_decode_launch(m->bf16, m->qkv, cl, m->y, B, H, C, c.n_ctx, pos + 1, s));
+    // the lm_head partials buffer is free until the end of the step: split-key scratch
+    G2_CK(attention_decode_launch(m->bf16, m->qkv, cl, m->y, B, H, C, c.n_ctx, pos + 1,
+                                  reinterpret_cast<float*>(m->part), (m->plan.tgt - m->plan.part) / sizeof(float), s));
     G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C,
                      m->x, C, s));
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));

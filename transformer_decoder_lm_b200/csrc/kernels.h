@@ -120,8 +120,11 @@ cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, 
 // softmax(q k^T / sqrt(D)) v with q from qkv [B, 3C] and k, v from one
 // layer's cache [max_B][n_ctx][2C] (k then v per position). D = C / H must
 // divide 128.
+// part: fp32 scratch of part_floats floats for the split-over-keys bf16
+// kernels (B * H * ceil(len / 256) * (D + 2) needed; otherwise, or when NULL,
+// one block per (sequence, head) takes all keys).
 cudaError_t attention_decode_launch(bool bf16, const void* qkv, const void* cache, void* y, int B, int H, int C,
-                                    int n_ctx, int len, cudaStream_t s);
+                                    int n_ctx, int len, float* part, size_t part_floats, cudaStream_t s);
 
 // ---- cross-entropy finalisation -------------------------------------------
 // token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
