@@ -92,6 +92,8 @@ LINEAR_SHAPES = [
     (128, 200, 64),       # one m-tile, N tail inside a 64-column group
     (515, 776, 256),      # N tail past 768
     (64, 1600, 1600),     # partial m-tile only
+    (5, 2304, 768),       # a few rows: the one-warp-per-column path
+    (16, 776, 3072),      # its largest row count, N tail, long K
 ]
 
 

@@ -157,7 +157,9 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   a.status = m->status;
   a.gelu_tanh = (m->cfg.flags & GPT2_FLAG_GELU_TANH) ? 1 : 0;
   cudaError_t e;
-  if (m->bf16) {
+  if (m->bf16 && M <= GEMV_MAX_M) {   // a few rows (decoding): one warp per output column
+    e = gemv_bf16_launch(epi, A, W, a, s);
+  } else if (m->bf16) {
     const int bn = gemm_tc_pick_bn(M, N, m->num_sms, epi);
     e = gemm_tc_launch(epi, bn, *tmA, wmaps[bn_index(bn)], *tmC, a, m->num_sms, s);
   } else {
@@ -574,6 +576,8 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
                ? GPT2_OK
                : GPT2_ERR_CUDA;
   if (K % 64) return GPT2_ERR_UNSUPPORTED;
+  if (M <= GEMV_MAX_M)
+    return gemv_bf16_launch(epilogue, A, W, a, s) == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
   int sms = 0;
   int rc = device_setup(nullptr, &sms);
   if (rc != GPT2_OK) return rc;

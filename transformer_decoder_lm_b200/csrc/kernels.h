@@ -85,6 +85,12 @@ cudaError_t embed_launch(bool bf16, const int* ids, const void* wte, const void*
 cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const void* b, void* out, int M, int C,
                              cudaStream_t s);
 
+// ---- Linear layers for a few rows (bf16, M <= GEMV_MAX_M) -------------------
+// The epilogues EPI_BIAS / EPI_GELU / EPI_RESID of GemmArgs, one warp per
+// output column; A [M, K] and W [N, K] 16-byte aligned, K a multiple of 8.
+constexpr int GEMV_MAX_M = 16;
+cudaError_t gemv_bf16_launch(int epi, const void* A, const void* W, const GemmArgs& a, cudaStream_t s);
+
 // ---- sinusoidal position table (bf16 or fp32 [n_ctx, C]) -------------------
 cudaError_t sinusoidal_wpe_launch(bool bf16, void* wpe, int n_ctx, int C, cudaStream_t s);
 
