@@ -23,6 +23,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "decode.h"
 #include "kernels.h"
 
 namespace g2 {

@@ -11,6 +11,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "decode.h"
 #include "kernels.h"
 
 namespace g2 {

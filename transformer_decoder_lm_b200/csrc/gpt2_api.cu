@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "gpt2.h"
+#include "decode.h"
 #include "kernels.h"
 
 using namespace g2;

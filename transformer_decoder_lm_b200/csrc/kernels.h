@@ -85,12 +85,6 @@ cudaError_t embed_launch(bool bf16, const int* ids, const void* wte, const void*
 cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const void* b, void* out, int M, int C,
                              cudaStream_t s);
 
-// ---- Linear layers for a few rows (bf16, M <= GEMV_MAX_M) -------------------
-// The epilogues EPI_BIAS / EPI_GELU / EPI_RESID of GemmArgs, one warp per
-// output column; A [M, K] and W [N, K] 16-byte aligned, K a multiple of 8.
-constexpr int GEMV_MAX_M = 16;
-cudaError_t gemv_bf16_launch(int epi, const void* A, const void* W, const GemmArgs& a, cudaStream_t s);
-
 // ---- sinusoidal position table (bf16 or fp32 [n_ctx, C]) -------------------
 cudaError_t sinusoidal_wpe_launch(bool bf16, void* wpe, int n_ctx, int C, cudaStream_t s);
 
@@ -121,16 +115,6 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
                                 int* status, cudaStream_t s);
 cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C,
                              const AttnScratch* scratch, int* status, cudaStream_t s);
-
-// One query per (sequence, head) against `len` cached positions: y [B, C] =
-// softmax(q k^T / sqrt(D)) v with q from qkv [B, 3C] and k, v from one
-// layer's cache [max_B][n_ctx][2C] (k then v per position). D = C / H must
-// divide 128.
-// part: fp32 scratch of part_floats floats for the split-over-keys bf16
-// kernels (B * H * ceil(len / 256) * (D + 2) needed; otherwise, or when NULL,
-// one block per (sequence, head) takes all keys).
-cudaError_t attention_decode_launch(bool bf16, const void* qkv, const void* cache, void* y, int B, int H, int C,
-                                    int n_ctx, int len, float* part, size_t part_floats, cudaStream_t s);
 
 // ---- cross-entropy finalisation -------------------------------------------
 // token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
