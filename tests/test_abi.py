@@ -48,6 +48,11 @@ def test_workspace_bytes_and_config_checks():
     ]
     for c in bad:
         assert B.gpt2_workspace_bytes(c, 1, 1) == 0
+    # key/value cache: [n_layer][max_B][n_ctx][2C] elements of the dtype
+    assert B.gpt2_kv_cache_bytes(ok, 4) == 12 * 4 * 1024 * 2 * 768 * 2
+    f32 = B.make_config(2, 2, 64, 512, 32, B.GPT2_FP32)
+    assert B.gpt2_kv_cache_bytes(f32, 3) == 2 * 3 * 32 * 2 * 64 * 4
+    assert B.gpt2_kv_cache_bytes(ok, 0) == 0 and B.gpt2_kv_cache_bytes(bad[0], 1) == 0
     # flags: the tanh-GELU bit is accepted, any other bit rejected
     assert B.gpt2_workspace_bytes(B.make_config(12, 12, 768, 50257, 1024, B.GPT2_BF16, B.GPT2_FLAG_GELU_TANH), 4, 1024) == n
     assert B.gpt2_workspace_bytes(B.make_config(12, 12, 768, 50257, 1024, B.GPT2_BF16, 2), 4, 1024) == 0
