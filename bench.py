@@ -207,13 +207,15 @@ def run_reference(args):
     v = args.steps * n / elapsed
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000.0 * WL.batch * WL.seq / v, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * elapsed / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WL.name, "global_batch": WL.batch * args.gpus, "seq_len": WL.seq,
                    "parallelism": f"dp{args.gpus}", "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": int(cores), "kind": "oracle",
                          "sample": f"per step the first {n} tokens of one 1024-token sequence of the 124M workload, "
-                                   f"fp64 NumPy forward + shifted cross-entropy ({elapsed:.1f} s over {args.steps} steps)"},
+                                   f"fp64 NumPy forward + shifted cross-entropy ({elapsed:.1f} s over {args.steps} steps); "
+                                   f"ms_per_step is the time of one such {n}-token step; a whole {WL.batch}x{WL.seq} "
+                                   f"batch would take {WL.batch * WL.seq / n:.1f} times as long"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -266,11 +268,6 @@ def run_ours(args):
     if rc != 0:
         raise RuntimeError(f"device status after warm-up: {G.gpt2_error_string(rc)}")
 
-    # per-launch timing of the dominant kernel (lm_head + fused CE) inside the timed steps
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for ev in ev_b + ev_e:   # creates the underlying CUDA events before their handles are passed on
-        ev.record(stream)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     launches0 = G.gpt2_launch_count(model.handle)
@@ -278,13 +275,27 @@ def run_ours(args):
     with ClockSampler(local) as clocks:
         t0.record(stream)
         for i in range(args.steps):
-            G.gpt2_set_timing_events(model.handle, G.binding.GPT2_TIMED_LMHEAD, ev_b[i], ev_e[i])
             step(ids, tg)
         t1.record(stream)
         barrier()
-    G.gpt2_set_timing_events(model.handle, G.binding.GPT2_TIMED_LMHEAD, None, None)
     launches = G.gpt2_launch_count(model.handle) - launches0
     ms = t0.elapsed_time(t1)
+
+    # The dominant kernel (lm_head + fused log-sum-exp) on a separate pass of
+    # the same steps, with CUDA events recorded around its launch on the
+    # launching stream (events between two kernels break their programmatic
+    # overlap, so they stay out of the step timing above).
+    lm_steps = min(args.steps, 50)
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(lm_steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(lm_steps)]
+    for ev in ev_b + ev_e:   # creates the underlying CUDA events before their handles are passed on
+        ev.record(stream)
+    barrier()
+    for i in range(lm_steps):
+        G.gpt2_set_timing_events(model.handle, G.binding.GPT2_TIMED_LMHEAD, ev_b[i], ev_e[i])
+        step(ids, tg)
+    G.gpt2_set_timing_events(model.handle, G.binding.GPT2_TIMED_LMHEAD, None, None)
+    barrier()
     lm_ms = float(np.mean([b.elapsed_time(e) for b, e in zip(ev_b, ev_e)]))
     rc = model.status()
     if rc != 0:
@@ -338,10 +349,11 @@ def run_ours(args):
         "frac_of_bf16_peak": total_tflops / tf_burst,
         "peak_note": f"{peak_kind} bf16 {tf_burst} TF/s burst, {tf_sust} sustained",
         "roofline": {"kernel": "lm_head tcgen05 GEMM + fused log-sum-exp (gemm_tc_kernel EPI_LMHEAD)",
-                     "bound": "tensor", "achieved": lm_tflops, "peak": tf_sust, "unit": "TFLOP/s",
-                     "frac": lm_tflops / tf_sust, "traffic": lmhead_traffic(),
+                     "bound": "tensor", "achieved": lm_tflops, "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": lm_tflops / tf_burst, "traffic": lmhead_traffic(),
                      "flops_per_launch": lmhead_flops(WL, M), "ms_per_launch": lm_ms,
-                     "peak_kind": f"{peak_kind} sustained (kernel timed inside a long step)"},
+                     "launches_timed": lm_steps,
+                     "peak_kind": f"{peak_kind} burst (the timed region lasts tens of milliseconds)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h_ids.numel() * 4 + h_tg.numel() * 4),
                 "d2h_bytes_per_step": 4},
         "gpu_launches": int(launches),
@@ -392,6 +404,12 @@ def run_kernel(args):
         qkv, y = rnd(M, 3 * C), torch.empty(M, C, dtype=bf, device="cuda")
         fn = lambda: G.gpt2_op_attention(G.GPT2_BF16, qkv, WL.batch, WL.seq, H, C, y)
         flops = WL.batch * 2.0 * C * WL.seq * (WL.seq + 1)
+    elif k == "embed":
+        ids = torch.from_numpy(rng.integers(0, V, size=M).astype(np.int32)).cuda()
+        wte, wpe = rnd(V, C, scale=0.02), rnd(WL.n_ctx, C, scale=0.02)
+        x = torch.empty(M, C, dtype=torch.float32, device="cuda")
+        fn = lambda: G.gpt2_op_embed(G.GPT2_BF16, ids, wte, wpe, M, WL.seq, C, V, x)
+        flops = 0.0
     elif k == "layernorm":
         x, g, b = rnd(M, C, dtype=torch.float32), rnd(C), rnd(C)
         out = torch.empty(M, C, dtype=bf, device="cuda")
@@ -453,7 +471,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None,
                     help="run one step alone: lmhead, lmhead_ce (no logits), c_attn, attn_proj, c_fc, mlp_proj, "
-                         "attention, layernorm, decode (one key/value-cache decoding step, B 4, context 1024)")
+                         "attention, embed, layernorm, decode (one key/value-cache decoding step, B 4, context 1024)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)

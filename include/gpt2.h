@@ -209,21 +209,24 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
  * Cache layout, `dtype` elements: [n_layer][max_B][n_ctx][2C], position t of
  * sequence b of layer l holding k (C values, heads concatenated) then v (C
  * values). max_B is the one given to gpt2_create; the caller allocates the
- * cache (gpt2_kv_cache_bytes, 0 for a bad config) and owns it. */
+ * cache (gpt2_kv_cache_bytes with that max_B, 0 for a bad config) and owns
+ * it. Both calls below take the cache's size in bytes and return
+ * GPT2_ERR_WORKSPACE, before any launch, when it is smaller than the layout
+ * of the handle needs (a cache sized for a smaller max_B than the handle's). */
 size_t gpt2_kv_cache_bytes(const gpt2_config_t* cfg, int max_B);
 
 /* The forward pass of gpt2_forward over ids [B, T] that also stores every
- * layer's k and v of positions 0..T-1 of each sequence in the cache.
- * logits_or_null as in gpt2_forward. */
-int gpt2_prefill(gpt2_handle_t h, void* kv_cache, const int32_t* ids, int B, int T,
+ * layer's k and v of positions 0..T-1 of each sequence in the cache of
+ * kv_bytes bytes. logits_or_null as in gpt2_forward. */
+int gpt2_prefill(gpt2_handle_t h, void* kv_cache, size_t kv_bytes, const int32_t* ids, int B, int T,
                  float* logits_or_null, void* stream);
 
 /* One new token per sequence at position pos (0 <= pos < n_ctx): ids_new
- * int32 [B]; the cache must hold positions 0..pos-1 of these B sequences
- * (from gpt2_prefill or earlier steps). Stores the new position's k and v in
- * the cache and writes logits fp32 [B, vocab] of the new position.
+ * int32 [B]; the cache (kv_bytes bytes) must hold positions 0..pos-1 of these
+ * B sequences (from gpt2_prefill or earlier steps). Stores the new position's
+ * k and v in the cache and writes logits fp32 [B, vocab] of the new position.
  * GPT2_ERR_UNSUPPORTED if pos >= n_ctx; GPT2_ERR_INVALID_ARG if B > max_B. */
-int gpt2_decode_step(gpt2_handle_t h, void* kv_cache, const int32_t* ids_new, int B, int pos,
+int gpt2_decode_step(gpt2_handle_t h, void* kv_cache, size_t kv_bytes, const int32_t* ids_new, int B, int pos,
                      float* logits, void* stream);
 
 /* Fixed sinusoidal position table ("Hand-writing GPT-2 from scratch: the

@@ -75,5 +75,12 @@ def test_decode_from_empty_cache_and_errors(G):
         model.decode_step(d_ids[:, 0].contiguous(), wl.n_ctx, cache)          # pos >= n_ctx
     with pytest.raises(G.GPT2Error):
         model.decode_step(torch.zeros(wl.batch + 1, dtype=torch.int32, device="cuda"), 1, cache)   # B > max_B
+    # a cache sized for fewer sequences than the handle's max_B is refused on the host
+    small = torch.empty(G.gpt2_kv_cache_bytes(model.cfg, wl.batch - 1), dtype=torch.uint8, device="cuda")
+    for call in (lambda: model.decode_step(d_ids[:, 0].contiguous(), 0, small),
+                 lambda: model.prefill(d_ids[:, :4].contiguous(), small, want_logits=False)):
+        with pytest.raises(G.GPT2Error) as e:
+            call()
+        assert e.value.code == G.binding.ERR_CODE["GPT2_ERR_WORKSPACE"]
     assert model.status() == 0
     model.close()

@@ -68,8 +68,8 @@ def _load():
         "gpt2_forward_loss": (i, [vp, vp, vp, i, i, vp, vp, vp, vp]),
         "gpt2_status": (i, [vp, vp]),
         "gpt2_kv_cache_bytes": (sz, [ctypes.POINTER(gpt2_config_t), i]),
-        "gpt2_prefill": (i, [vp, vp, vp, i, i, vp, vp]),
-        "gpt2_decode_step": (i, [vp, vp, vp, i, i, vp, vp]),
+        "gpt2_prefill": (i, [vp, vp, sz, vp, i, i, vp, vp]),
+        "gpt2_decode_step": (i, [vp, vp, sz, vp, i, i, vp, vp]),
         "gpt2_error_string": (ctypes.c_char_p, [i]),
         "gpt2_destroy": (None, [vp]),
         "gpt2_launch_count": (ctypes.c_uint64, [vp]),
@@ -162,13 +162,18 @@ def gpt2_kv_cache_bytes(cfg: gpt2_config_t, max_B: int) -> int:
     return int(lib.gpt2_kv_cache_bytes(ctypes.byref(cfg), max_B))
 
 
+def _nbytes(t) -> int:
+    return 0 if t is None else int(t.numel() * t.element_size())
+
+
 def gpt2_prefill(h, kv_cache, ids, B: int, T: int, logits=None, stream=None) -> None:
-    _check(lib.gpt2_prefill(h, _ptr(kv_cache), _ptr(ids), B, T, _ptr(logits), _stream(stream)), "gpt2_prefill")
+    _check(lib.gpt2_prefill(h, _ptr(kv_cache), _nbytes(kv_cache), _ptr(ids), B, T, _ptr(logits), _stream(stream)),
+           "gpt2_prefill")
 
 
 def gpt2_decode_step(h, kv_cache, ids_new, B: int, pos: int, logits, stream=None) -> None:
-    _check(lib.gpt2_decode_step(h, _ptr(kv_cache), _ptr(ids_new), B, pos, _ptr(logits), _stream(stream)),
-           "gpt2_decode_step")
+    _check(lib.gpt2_decode_step(h, _ptr(kv_cache), _nbytes(kv_cache), _ptr(ids_new), B, pos, _ptr(logits),
+                                _stream(stream)), "gpt2_decode_step")
 
 
 def gpt2_status(h, stream=None) -> int:

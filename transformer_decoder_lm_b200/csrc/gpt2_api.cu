@@ -478,16 +478,18 @@ size_t gpt2_kv_cache_bytes(const gpt2_config_t* cfg, int max_B) {
   return (size_t)cfg->n_layer * max_B * cfg->n_ctx * 2 * cfg->n_embd * es;
 }
 
-int gpt2_prefill(gpt2_handle_t h, void* kv_cache, const int32_t* ids, int B, int T, float* logits_or_null,
-                 void* stream) {
-  if (!kv_cache || !aligned16(kv_cache)) return GPT2_ERR_INVALID_ARG;
+int gpt2_prefill(gpt2_handle_t h, void* kv_cache, size_t kv_bytes, const int32_t* ids, int B, int T,
+                 float* logits_or_null, void* stream) {
+  if (!h || !kv_cache || !aligned16(kv_cache)) return GPT2_ERR_INVALID_ARG;
+  if (kv_bytes < (size_t)h->cfg.n_layer * kv_layer_bytes(h)) return GPT2_ERR_WORKSPACE;
   return run_forward(h, ids, nullptr, B, T, logits_or_null, nullptr, nullptr, static_cast<cudaStream_t>(stream),
                      kv_cache);
 }
 
-int gpt2_decode_step(gpt2_handle_t h, void* kv_cache, const int32_t* ids_new, int B, int pos, float* logits,
-                     void* stream) {
-  if (!kv_cache || !aligned16(kv_cache)) return GPT2_ERR_INVALID_ARG;
+int gpt2_decode_step(gpt2_handle_t h, void* kv_cache, size_t kv_bytes, const int32_t* ids_new, int B, int pos,
+                     float* logits, void* stream) {
+  if (!h || !kv_cache || !aligned16(kv_cache)) return GPT2_ERR_INVALID_ARG;
+  if (kv_bytes < (size_t)h->cfg.n_layer * kv_layer_bytes(h)) return GPT2_ERR_WORKSPACE;
   return run_decode(h, kv_cache, ids_new, B, pos, logits, static_cast<cudaStream_t>(stream));
 }
 

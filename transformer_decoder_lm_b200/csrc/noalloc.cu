@@ -18,6 +18,7 @@
 // (on different streams, or from different host threads) race on it; keep
 // them ordered. Nothing in the array has to start at zero: every partial
 // that the finishing kernel reads is written earlier in the same call.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -102,7 +103,7 @@ extern "C" int gpt2_op_lmhead_ce_noalloc(int dtype, const void* hf, const void* 
   a.status = status;
   int n_groups;
   if (dtype == GPT2_BF16) {
-    const int bn = gemm_tc_pick_bn(M, V, d->num_sms, EPI_LMHEAD) < LMHEAD_MIN_BN ? LMHEAD_MIN_BN : gemm_tc_pick_bn(M, V, d->num_sms, EPI_LMHEAD);
+    const int bn = std::max(gemm_tc_pick_bn(M, V, d->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
     n_groups = gemm_tc_n_tiles(V, bn);
     CUtensorMap ta, tb;
     if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;

@@ -5,7 +5,7 @@ its own batch of B sequences through the C ABI; no activation crosses GPUs.
 The only exchange is the loss: the mean over all ranks' scored positions
 needs the sum of per-position losses and their count from every rank, one
 all-reduce of two numbers ("Hand-writing GPT-2 from scratch: the Transformer
-decoder core modules in PyTorch", section 5: the DDP set-up with the NCCL
+decoder core modules in PyTorch", section 6.2: the DDP set-up with the NCCL
 backend; here only the forward's loss is combined).
 """
 from __future__ import annotations
