@@ -1,6 +1,7 @@
-"""GPT-2 decoder forward pass on one B200 (sm_100a).
+"""GPT-2 decoder forward and backward passes on one B200 (sm_100a).
 
-The product is the C-ABI library libgpt2.so (include/gpt2.h) built from
+The product is the C-ABI library libgpt2.so (include/gpt2.h,
+include/gpt2_train.h) built from
 csrc/; ``binding`` is its ctypes binding (same names as the C entry points)
 and ``model.GPT2Model`` a small owner of device weights, workspace and
 handle. Importing this package fails if libgpt2.so has not been built.
@@ -15,5 +16,9 @@ from .binding import (  # noqa: F401
     gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear,
     gpt2_op_attention, gpt2_op_lmhead_ce_workspace_bytes, gpt2_op_lmhead_ce, make_config,
     gpt2_op_lmhead_ce_noalloc, GPT2_NOALLOC_SCRATCH_BYTES,
+    gpt2_train_workspace_bytes, gpt2_forward_backward, gpt2_op_linear_dgrad, gpt2_op_linear_wgrad,
+    gpt2_op_linear_dgrad_gelu, gpt2_op_layernorm_backward_workspace_bytes, gpt2_op_layernorm_backward,
+    gpt2_op_attention_train, gpt2_op_attention_backward_workspace_bytes, gpt2_op_attention_backward,
+    gpt2_op_lmhead_ce_backward_workspace_bytes, gpt2_op_lmhead_ce_backward,
 )
 from .model import GPT2Model, upload_weights  # noqa: F401

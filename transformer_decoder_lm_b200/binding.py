@@ -54,6 +54,12 @@ class gpt2_weights_t(ctypes.Structure):
                [("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p)]
 
 
+class gpt2_grads_t(ctypes.Structure):
+    _fields_ = [("wte", ctypes.c_void_p), ("wpe", ctypes.c_void_p)] + \
+               [(k, _PP) for k in LAYER_KEYS] + \
+               [("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libgpt2.so is not built ({LIB_PATH}); run python transformer_decoder_lm_b200/build.py")
@@ -82,6 +88,19 @@ def _load():
         "gpt2_op_lmhead_ce_workspace_bytes": (sz, [i, i, i]),
         "gpt2_op_lmhead_ce": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
         "gpt2_op_lmhead_ce_noalloc": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, vp]),
+        # include/gpt2_train.h
+        "gpt2_train_workspace_bytes": (sz, [ctypes.POINTER(gpt2_config_t), i, i]),
+        "gpt2_forward_backward": (i, [vp, vp, vp, i, i, vp, ctypes.POINTER(gpt2_grads_t), vp, sz, vp]),
+        "gpt2_op_linear_dgrad": (i, [vp, vp, i, i, i, vp, i, vp, vp]),
+        "gpt2_op_linear_wgrad": (i, [vp, vp, i, i, i, vp, vp, vp]),
+        "gpt2_op_linear_dgrad_gelu": (i, [vp, vp, vp, i, i, i, i, vp, vp, vp]),
+        "gpt2_op_layernorm_backward_workspace_bytes": (sz, [i, i]),
+        "gpt2_op_layernorm_backward": (i, [vp, vp, vp, vp, i, i, vp, vp, vp, vp, sz, vp]),
+        "gpt2_op_attention_train": (i, [vp, i, i, i, i, vp, vp, vp, vp]),
+        "gpt2_op_attention_backward_workspace_bytes": (sz, [i, i, i, i]),
+        "gpt2_op_attention_backward": (i, [vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]),
+        "gpt2_op_lmhead_ce_backward_workspace_bytes": (sz, [i, i]),
+        "gpt2_op_lmhead_ce_backward": (i, [vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -246,3 +265,79 @@ def gpt2_op_lmhead_ce_noalloc(dtype, hf, wte, targets, M, C, V, logits, token_lo
     _check(lib.gpt2_op_lmhead_ce_noalloc(dtype, _ptr(hf), _ptr(wte), _ptr(targets), M, C, V, _ptr(logits),
                                          _ptr(token_loss), _ptr(loss_out), _ptr(status), _stream(stream)),
            "gpt2_op_lmhead_ce_noalloc")
+
+
+# ---- include/gpt2_train.h ---------------------------------------------------
+
+def gpt2_train_workspace_bytes(cfg: gpt2_config_t, max_B: int, max_T: int) -> int:
+    return int(lib.gpt2_train_workspace_bytes(ctypes.byref(cfg), max_B, max_T))
+
+
+class _Grads:
+    """Keeps the ctypes pointer arrays of a gradient dict alive (layout of the
+    weights dict: 'wte', 'wpe', 'lnf_g', 'lnf_b', 'layers': [{LAYER_KEYS}])."""
+
+    def __init__(self, g: Dict[str, object]):
+        n = len(g["layers"])
+        self.arrays = {k: (ctypes.c_void_p * n)(*[_ptr(lg[k]) for lg in g["layers"]]) for k in LAYER_KEYS}
+        self.struct = gpt2_grads_t(
+            _ptr(g["wte"]), _ptr(g["wpe"]),
+            *[ctypes.cast(self.arrays[k], _PP) for k in LAYER_KEYS],
+            _ptr(g["lnf_g"]), _ptr(g["lnf_b"]))
+
+
+def gpt2_forward_backward(h, ids, targets, B: int, T: int, loss_out, grads: Dict[str, object], train_ws,
+                          stream=None) -> None:
+    keep = _Grads(grads)
+    _check(lib.gpt2_forward_backward(h, _ptr(ids), _ptr(targets), B, T, _ptr(loss_out), ctypes.byref(keep.struct),
+                                     _ptr(train_ws), _nbytes(train_ws), _stream(stream)), "gpt2_forward_backward")
+
+
+def gpt2_op_linear_dgrad(dy, W, M, N, K, dx, out_f32=True, status=None, stream=None):
+    _check(lib.gpt2_op_linear_dgrad(_ptr(dy), _ptr(W), M, N, K, _ptr(dx), int(bool(out_f32)), _ptr(status),
+                                    _stream(stream)), "gpt2_op_linear_dgrad")
+
+
+def gpt2_op_linear_wgrad(dy, x, M, N, K, dW, status=None, stream=None):
+    _check(lib.gpt2_op_linear_wgrad(_ptr(dy), _ptr(x), M, N, K, _ptr(dW), _ptr(status), _stream(stream)),
+           "gpt2_op_linear_wgrad")
+
+
+def gpt2_op_linear_dgrad_gelu(dy, W, u, M, N, K, tanh_form, du, status=None, stream=None):
+    _check(lib.gpt2_op_linear_dgrad_gelu(_ptr(dy), _ptr(W), _ptr(u), M, N, K, int(tanh_form), _ptr(du), _ptr(status),
+                                         _stream(stream)), "gpt2_op_linear_dgrad_gelu")
+
+
+def gpt2_op_layernorm_backward_workspace_bytes(M, C) -> int:
+    return int(lib.gpt2_op_layernorm_backward_workspace_bytes(M, C))
+
+
+def gpt2_op_layernorm_backward(x, gamma, dh, dx_in, M, C, dx_out, dgamma, dbeta, workspace, stream=None):
+    _check(lib.gpt2_op_layernorm_backward(_ptr(x), _ptr(gamma), _ptr(dh), _ptr(dx_in), M, C, _ptr(dx_out),
+                                          _ptr(dgamma), _ptr(dbeta), _ptr(workspace), _nbytes(workspace),
+                                          _stream(stream)), "gpt2_op_layernorm_backward")
+
+
+def gpt2_op_attention_train(qkv, B, T, H, C, y, lse2, status=None, stream=None):
+    _check(lib.gpt2_op_attention_train(_ptr(qkv), B, T, H, C, _ptr(y), _ptr(lse2), _ptr(status), _stream(stream)),
+           "gpt2_op_attention_train")
+
+
+def gpt2_op_attention_backward_workspace_bytes(B, T, H, C) -> int:
+    return int(lib.gpt2_op_attention_backward_workspace_bytes(B, T, H, C))
+
+
+def gpt2_op_attention_backward(qkv, y, dy, lse2, B, T, H, C, dqkv, workspace, stream=None):
+    _check(lib.gpt2_op_attention_backward(_ptr(qkv), _ptr(y), _ptr(dy), _ptr(lse2), B, T, H, C, _ptr(dqkv),
+                                          _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "gpt2_op_attention_backward")
+
+
+def gpt2_op_lmhead_ce_backward_workspace_bytes(M, V) -> int:
+    return int(lib.gpt2_op_lmhead_ce_backward_workspace_bytes(M, V))
+
+
+def gpt2_op_lmhead_ce_backward(hf, wte, targets, M, C, V, loss_out, dhf, dwte, workspace, status=None, stream=None):
+    _check(lib.gpt2_op_lmhead_ce_backward(_ptr(hf), _ptr(wte), _ptr(targets), M, C, V, _ptr(loss_out), _ptr(dhf),
+                                          _ptr(dwte), _ptr(workspace), _nbytes(workspace), _ptr(status),
+                                          _stream(stream)), "gpt2_op_lmhead_ce_backward")

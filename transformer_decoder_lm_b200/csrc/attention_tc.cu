@@ -155,7 +155,7 @@ template <bool kSplit>
 __global__ void __launch_bounds__(AT_THREADS, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_y, int B,
                        int T, int H, int C, float scale_log2, const __grid_constant__ AttnPlan plan,
-                       unsigned* sched, int* flags, float* part, int n_flags, int* status) {
+                       unsigned* sched, int* flags, float* part, int n_flags, int* status, float* lse_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;      // [2]
@@ -523,6 +523,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         continue;
       }
       float fa = 0.f, fb = 1.f / l;
+      float lse2 = m + __log2f(l);   // log2 of the softmax normaliser, in the units of scale_log2 * s
       bool own_first = false;
       const float* pb = part + (size_t)w.pair * ATTN_PART_FLOATS;
       if (kSplit && merge) {   // merge with the other half's partial rows
@@ -545,7 +546,9 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         const float inv = 1.f / (l1 * a1 + l2 * a2);
         fa = a1 * inv;   // factor of range (1)
         fb = a2 * inv;   // factor of range (2)
+        lse2 = mx + __log2f(l1 * a1 + l2 * a2);
       }
+      if (lse_out != nullptr && i < T) lse_out[((size_t)b * H + h) * T + i] = lse2;
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -698,7 +701,7 @@ size_t attention_scratch_bytes(int B, int T, int H) {
 }
 
 cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, const AttnScratch* scratch,
-                                int* status, cudaStream_t s) {
+                                int* status, cudaStream_t s, float* lse_out) {
   if (B <= 0 || T <= 0) return cudaSuccess;
   if (C / H != AT_D) return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
@@ -745,15 +748,16 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
   const int QT = (T + AT_BQ - 1) / AT_BQ;
   const int BH = B * H;
   int n_split = 0;
-  const AttnPlan plan = make_plan(BH, QT, slots[dev], sc.flags && sc.part ? sc.cap_pairs : 0, &n_split);
+  const AttnPlan plan =
+      make_plan(BH, QT, slots[dev], (sc.flags && sc.part && lse_out == nullptr) ? sc.cap_pairs : 0, &n_split);
   const int items = BH * (plan.n_cls ? plan.n_cls : QT);
   const int grid = items < slots[dev] ? items : slots[dev];
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)AT_D));
   if (n_split)
     return launch_pdl(attn_fwd_tc_kernel<true>, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
-                      plan, sc.sched, sc.flags, sc.part, n_split * BH * ATTN_PAIR_FLAGS, status);
+                      plan, sc.sched, sc.flags, sc.part, n_split * BH * ATTN_PAIR_FLAGS, status, lse_out);
   return launch_pdl(attn_fwd_tc_kernel<false>, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
-                    plan, sc.sched, sc.flags, sc.part, 0, status);
+                    plan, sc.sched, sc.flags, sc.part, 0, status, lse_out);
 }
 
 }  // namespace g2

@@ -33,7 +33,8 @@ __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2
 __global__ void __launch_bounds__(32 * CE_WARPS) ce_rows_kernel(const float2* __restrict__ part, int n_tiles,
                                                                const float* __restrict__ tgt_logit,
                                                                const int* __restrict__ targets, int M, int V,
-                                                               float* __restrict__ token_loss, int* status) {
+                                                               float* __restrict__ token_loss, int* status,
+                                                               float* __restrict__ lse_out) {
   __shared__ float sm_m[CE_WARPS][32], sm_s[CE_WARPS][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 32 + lane;
@@ -66,6 +67,7 @@ __global__ void __launch_bounds__(32 * CE_WARPS) ce_rows_kernel(const float2* __
     for (int w = 0; w < CE_WARPS; ++w) lse_merge(mm, ss, sm_m[w][lane], sm_s[w][lane]);
     const int tg = targets[row];
     float l = 0.f;
+    if (lse_out) lse_out[row] = mm + logf(ss);
     if (tg >= V) {
       record_error(status, DEV_BAD_TOKEN);
     } else if (tg >= 0) {
@@ -77,7 +79,8 @@ __global__ void __launch_bounds__(32 * CE_WARPS) ce_rows_kernel(const float2* __
 
 __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__ token_loss,
                                                        const int* __restrict__ targets, int M, int V,
-                                                       float* __restrict__ loss_out, int* status) {
+                                                       float* __restrict__ loss_out, int* status,
+                                                       int* __restrict__ n_scored_out) {
   __shared__ double ssum[32];
   __shared__ int scnt[32];
   pdl_wait();
@@ -112,6 +115,7 @@ __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__
       cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
     }
     if (lane == 0) {
+      if (n_scored_out) *n_scored_out = cnt;
       if (cnt == 0) {
         record_error(status, DEV_NO_TARGETS);
         *loss_out = __int_as_float(0x7fc00000);
@@ -123,12 +127,14 @@ __global__ void __launch_bounds__(1024) ce_mean_kernel(const float* __restrict__
 }
 
 cudaError_t ce_finish_launch(const float2* part, int n_tiles, const float* tgt_logit, const int* targets, int M,
-                             int V, float* token_loss, float* loss_out, int* status, cudaStream_t s) {
+                             int V, float* token_loss, float* loss_out, int* status, cudaStream_t s, float* lse_out,
+                             int* n_scored_out) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = launch_pdl(ce_rows_kernel, dim3((M + 31) / 32), dim3(32 * CE_WARPS), 0, s, part, n_tiles, tgt_logit, targets,
-                             M, V, token_loss, status);
+                             M, V, token_loss, status, lse_out);
   if (e == cudaSuccess && loss_out)
-    e = launch_pdl(ce_mean_kernel, dim3(1), dim3(1024), 0, s, token_loss, targets, M, V, loss_out, status);
+    e = launch_pdl(ce_mean_kernel, dim3(1), dim3(1024), 0, s, token_loss, targets, M, V, loss_out, status,
+                   n_scored_out);
   return e;
 }
 

@@ -274,6 +274,26 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Instruction descriptor of tcgen05.mma kind::f16 (bf16 in, fp32 D) with
+// either operand K-major (false) or MN-major (true).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+}
+
+// Shared-memory descriptor for an MN-major operand tile with 128-byte swizzle
+// made of 64-element MN blocks (one TMA box of 64 MN elements x K rows each),
+// the blocks `block_bytes` apart: rows of 128 B along K, 8-row groups 1024 B
+// apart; the start advances 2048 B per 16 K rows.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t block_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);           // start address
+  d |= (uint64_t)((block_bytes >> 4) & 0x3FFFu) << 16; // leading byte offset: next 64-wide MN block
+  d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset: next 8 rows of K
+  d |= (uint64_t)1 << 46;                             // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                             // 128-byte swizzle
+  return d;
+}
+
 // ------------------------------------------------------------------ math
 // 2^x with the SFU's approximate exponential (relative error about 2^-22,
 // results below 2^-126 flushed to zero; 2^-inf = 0).

@@ -80,10 +80,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // C <= 32 lanes * 4 * MAXV = 2048.
+// x_save (training forward): if not NULL, also receives a copy of x, the
+// LayerNorm input the backward pass differentiates at.
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(128) layernorm_kernel(const float* __restrict__ x, const T* __restrict__ g,
                                                         const T* __restrict__ b, T* __restrict__ out, int M,
-                                                        int C) {
+                                                        int C, float* __restrict__ x_save) {
   const int warps = blockDim.x >> 5;
   const int row = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -111,6 +113,14 @@ __global__ void __launch_bounds__(128) layernorm_kernel(const float* __restrict_
   for (int i = 0; i < MAXV; ++i) {
     const int c = (lane + 32 * i) * 4;
     if (c < C) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  }
+  if (x_save != nullptr) {
+    float* xs = x_save + (size_t)row * C;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int c = (lane + 32 * i) * 4;
+      if (c < C) Vec4<float>::store(xs + c, v[i]);
+    }
   }
   const float mean = warp_sum(s) / (float)C;
   float q = 0.f;
@@ -156,7 +166,7 @@ cudaError_t embed_launch(bool bf16_, const int* ids, const void* wte, const void
 }
 
 cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const void* b, void* out, int M, int C,
-                             cudaStream_t s) {
+                             cudaStream_t s, float* x_save) {
   if (M <= 0) return cudaSuccess;
   if (C > 2048 || (C & 3)) return cudaErrorInvalidValue;
   const int threads = 128, rows_per_block = threads / 32;
@@ -165,19 +175,19 @@ cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const vo
     // registers per lane grow with C: pick the smallest row capacity that fits
     const bf16 *gp = static_cast<const bf16*>(g), *bp = static_cast<const bf16*>(b);
     bf16* op = static_cast<bf16*>(out);
-    if (C <= 768) return launch_pdl(layernorm_kernel<bf16, 6>, grid, threads, 0, s, x, gp, bp, op, M, C);
-    if (C <= 1024) return launch_pdl(layernorm_kernel<bf16, 8>, grid, threads, 0, s, x, gp, bp, op, M, C);
-    if (C <= 1280) return launch_pdl(layernorm_kernel<bf16, 10>, grid, threads, 0, s, x, gp, bp, op, M, C);
-    if (C <= 1664) return launch_pdl(layernorm_kernel<bf16, 13>, grid, threads, 0, s, x, gp, bp, op, M, C);
-    return launch_pdl(layernorm_kernel<bf16, 16>, grid, threads, 0, s, x, gp, bp, op, M, C);
+    if (C <= 768) return launch_pdl(layernorm_kernel<bf16, 6>, grid, threads, 0, s, x, gp, bp, op, M, C, x_save);
+    if (C <= 1024) return launch_pdl(layernorm_kernel<bf16, 8>, grid, threads, 0, s, x, gp, bp, op, M, C, x_save);
+    if (C <= 1280) return launch_pdl(layernorm_kernel<bf16, 10>, grid, threads, 0, s, x, gp, bp, op, M, C, x_save);
+    if (C <= 1664) return launch_pdl(layernorm_kernel<bf16, 13>, grid, threads, 0, s, x, gp, bp, op, M, C, x_save);
+    return launch_pdl(layernorm_kernel<bf16, 16>, grid, threads, 0, s, x, gp, bp, op, M, C, x_save);
   } else {
     if (C <= 1024)
       layernorm_kernel<float, 8><<<grid, threads, 0, s>>>(x, static_cast<const float*>(g),
-                                                          static_cast<const float*>(b), static_cast<float*>(out), M, C);
+                                                          static_cast<const float*>(b), static_cast<float*>(out), M, C, x_save);
     else
       layernorm_kernel<float, 16><<<grid, threads, 0, s>>>(x, static_cast<const float*>(g),
                                                            static_cast<const float*>(b), static_cast<float*>(out), M,
-                                                           C);
+                                                           C, x_save);
   }
   return cudaGetLastError();
 }

@@ -63,7 +63,8 @@ struct TcLayout {
   static constexpr int THREADS = 32 * (2 + EPI_WARPS);
   // per epilogue warp: one 32 x 32 chunk (bf16: 2 KB, fp32 residual: 4 KB),
   // or 8 logits rows x 64 fp32 (2 KB)
-  static constexpr int STAGE_BUF_BYTES = EPI == EPI_RESID ? 4096 : 2048;
+  static constexpr bool F32_OUT = EPI == EPI_RESID || EPI == EPI_F32;
+  static constexpr int STAGE_BUF_BYTES = F32_OUT ? 4096 : 2048;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -78,14 +79,14 @@ struct TcLayout {
   static_assert(BN % COLS_PER_WARP == 0 && COLS_PER_WARP % 64 == 0, "whole 64-column groups per warp");
 };
 
-// Bias slice of one 32-column chunk (bf16 -> fp32 registers); zeros past N.
-// The same 32 bias values as bf16 pairs (lo = even column), zero past N.
+// The 32 bias values of one 32-column chunk as bf16 pairs (lo = even
+// column), zero past N or without a bias.
 __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int N, uint32_t (&b)[16]) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     const int col = col0 + g * 8;
     uint4 w = make_uint4(0, 0, 0, 0);
-    if (col < N) w = __ldg(reinterpret_cast<const uint4*>(bias + col));
+    if (bias != nullptr && col < N) w = __ldg(reinterpret_cast<const uint4*>(bias + col));
     b[4 * g] = w.x;
     b[4 * g + 1] = w.y;
     b[4 * g + 2] = w.z;
@@ -93,12 +94,27 @@ __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int 
   }
 }
 
-template <int BN, int EPI>
+// Derivative of the GELU at the pre-activation u: exact form
+// d/du [u Phi(u)] = Phi(u) + u phi(u); tanh form
+// d/du [u (1 + tanh(k (u + c u^3))) / 2] = (1 + t) / 2 + u (1 - t^2) k (1 + 3 c u^2) / 2.
+__device__ __forceinline__ float gelu_grad(float u, int tanh_form) {
+  if (tanh_form) {
+    const float k = 0.7978845608028654f, c = 0.044715f;
+    const float t = tanhf(k * fmaf(c * u * u, u, u));
+    return 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * k * fmaf(3.f * c, u * u, 1.f);
+  }
+  return 0.5f * (1.f + erff(u * 0.70710678118654752f)) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+}
+
+template <int BN, int EPI, int LAYOUT>
 __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                   const GemmArgs args) {
   using L = TcLayout<BN, EPI>;
   constexpr bool kLM = EPI == EPI_LMHEAD || EPI == EPI_LMHEAD_LOGITS;
+  constexpr bool kAmn = (LAYOUT & LAYOUT_A_MN) != 0, kBmn = (LAYOUT & LAYOUT_B_MN) != 0;
+  constexpr bool kGelu = EPI == EPI_GELU || EPI == EPI_GELU_SAVE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
@@ -115,7 +131,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   const int m_tiles = (M + TC_BM - 1) / TC_BM;
   const int n_tiles = (N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles;
-  const int nk = args.K / TC_BK;
+  const int nk = (args.K + TC_BK - 1) / TC_BK;   // a K tail past args.K reads as zero (TMA fill)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_STAGES; ++s) {
@@ -134,6 +150,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     if (!kLM) tma_prefetch_desc(&tmC);
+    if (EPI == EPI_GELU_SAVE) tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, L::TMEM_COLS);
@@ -162,8 +179,20 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           }
           uint8_t* sa = smem + stage * L::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &full[stage], kb * TC_BK, m0);
-          tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * TC_BK, n0);
+          // K-major: one box of rows x 64 K; MN-major: 64-wide MN boxes of 64 K rows, 8 KB apart
+          if (kAmn) {
+#pragma unroll
+            for (int b = 0; b < TC_BM / 64; ++b) tma_load_2d(sa + b * 8192, &tmA, &full[stage], m0 + b * 64, kb * TC_BK);
+          } else {
+            tma_load_2d(sa, &tmA, &full[stage], kb * TC_BK, m0);
+          }
+          if (kBmn) {
+#pragma unroll
+            for (int b = 0; b < BN / 64; ++b)
+              tma_load_2d(sa + L::A_BYTES + b * 8192, &tmB, &full[stage], n0 + b * 64, kb * TC_BK);
+          } else {
+            tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * TC_BK, n0);
+          }
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == TC_STAGES) {
@@ -184,7 +213,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, BN);
+      constexpr uint32_t IDESC = idesc_bf16_f32_major(TC_BM, BN, kAmn, kBmn);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -205,11 +234,14 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
-          const uint64_t adesc = sdesc_kmajor_sw128(sa);
-          const uint64_t bdesc = sdesc_kmajor_sw128(sa + L::A_BYTES);
 #pragma unroll
-          for (int k = 0; k < TC_BK / 16; ++k)
-            mma_bf16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0);
+          for (int k = 0; k < TC_BK / 16; ++k) {
+            // K step of 16: +32 B inside a K-major 128-byte row, +16 rows (2048 B) of an MN-major box
+            const uint64_t adesc = kAmn ? sdesc_mn_sw128(sa + k * 2048, 8192) : sdesc_kmajor_sw128(sa) + 2 * k;
+            const uint64_t bdesc =
+                kBmn ? sdesc_mn_sw128(sa + L::A_BYTES + k * 2048, 8192) : sdesc_kmajor_sw128(sa + L::A_BYTES) + 2 * k;
+            mma_bf16_ss(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
+          }
           mma_commit(&empty[stage]);
           if (++stage == TC_STAGES) {
             stage = 0;
@@ -353,10 +385,10 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           }
         }
       } else {
-        // bias / GELU / residual: both 32-column chunks of this warp's slice
-        // come out of TMEM with one wait and the accumulator goes straight
-        // back to the MMA warp; then per chunk: bias, activation, swizzled
-        // staging, TMA store or reduce-add.
+        // bias / GELU / residual / backward epilogues: both 32-column chunks
+        // of this warp's slice come out of TMEM with one wait and the
+        // accumulator goes straight back to the MMA warp; then per chunk:
+        // bias, activation, swizzled staging, TMA store or reduce-add.
         const int nch = (row0 < M && nvalid > 0) ? min(L::CHUNKS, (nvalid + 31) / 32) : 0;   // warp-uniform
         uint32_t v[L::CHUNKS][32];
 #pragma unroll
@@ -367,40 +399,24 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
         const bf16* bias_p = static_cast<const bf16*>(args.bias);
-#pragma unroll
-        for (int c = 0; c < L::CHUNKS; ++c) {
-          if (c >= nch) break;
-          const int col0 = cbase + c * 32;
-          uint32_t bc[16];   // bias as bf16 pairs
-          load_bias32_raw(bias_p, col0, N, bc);
-          uint32_t* pk = v[c];   // results overwrite the accumulator values in place
-          if (EPI == EPI_RESID) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              pk[2 * j] = __float_as_uint(__uint_as_float(v[c][2 * j]) + __uint_as_float(bc[j] << 16));
-              pk[2 * j + 1] = __float_as_uint(__uint_as_float(v[c][2 * j + 1]) + __uint_as_float(bc[j] & 0xffff0000u));
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float b0 = __uint_as_float(bc[j] << 16), b1 = __uint_as_float(bc[j] & 0xffff0000u);
-              const float x0 = __uint_as_float(v[c][2 * j]), x1 = __uint_as_float(v[c][2 * j + 1]);
-              if (EPI == EPI_GELU) {
-                const uint64_t z2 = f2_add(f2_pack(x0, x1), f2_pack(b0, b1));
-                const uint64_t y2 = args.gelu_tanh ? gelu_tanh_x2(z2) : gelu_erf_x2(z2);
-                float a, b;
-                f2_unpack(y2, a, b);
-                pk[j] = pack_bf16x2(a, b);
-              } else {
-                pk[j] = pack_bf16x2(x0 + b0, x1 + b1);
-              }
-            }
+        // EPI_DLOGITS: this row's target, log-sum-exp (log2 units) and 1 / scored rows
+        int d_tgt = -1;
+        float d_lse2 = 0.f, d_inv = 0.f;
+        if (EPI == EPI_DLOGITS) {
+          if (row_ok) {
+            d_tgt = args.targets[row];
+            d_lse2 = args.row_lse[row] * LOG2E;
           }
+          const int ns = *args.n_scored;
+          d_inv = ns > 0 ? 1.f / (float)ns : 0.f;
+        }
+        // stage 32 rows of one chunk in this warp's buffer and send it to `map`
+        auto stage_and_send = [&](const uint32_t* pk, const CUtensorMap* map, int col0) {
           if (store_pending) {       // the previous TMA store must have read the staging buffer
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
           }
-          if (EPI == EPI_RESID) {
+          if (L::F32_OUT) {
             // 32 rows x 128 B, 128-byte swizzle: unit j of row r at unit j ^ (r & 7)
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -417,12 +433,84 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           __syncwarp();
           if (lane == 0) {
             if (EPI == EPI_RESID)
-              tma_reduce_add_2d(&tmC, sbuf, col0, row0);
+              tma_reduce_add_2d(map, sbuf, col0, row0);
             else
-              tma_store_2d(&tmC, sbuf, col0, row0);
+              tma_store_2d(map, sbuf, col0, row0);
             bulk_commit();
           }
           store_pending = true;
+        };
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          if (c >= nch) break;
+          const int col0 = cbase + c * 32;
+          uint32_t* pk = v[c];   // results overwrite the accumulator values in place
+          if (L::F32_OUT) {
+            uint32_t bc[16];   // bias as bf16 pairs
+            load_bias32_raw(bias_p, col0, N, bc);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              pk[2 * j] = __float_as_uint(__uint_as_float(v[c][2 * j]) + __uint_as_float(bc[j] << 16));
+              pk[2 * j + 1] = __float_as_uint(__uint_as_float(v[c][2 * j + 1]) + __uint_as_float(bc[j] & 0xffff0000u));
+            }
+          } else if (EPI == EPI_DGELU) {
+            // dU = dF * gelu'(u) with u the saved pre-activation (bf16 pairs)
+            uint32_t ur[16];
+            const bf16* up = static_cast<const bf16*>(args.aux) + (size_t)row * args.ld_aux + col0;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint4 w = make_uint4(0, 0, 0, 0);
+              if (row_ok && col0 + g * 8 < N) w = __ldg(reinterpret_cast<const uint4*>(up + g * 8));
+              ur[4 * g] = w.x;
+              ur[4 * g + 1] = w.y;
+              ur[4 * g + 2] = w.z;
+              ur[4 * g + 3] = w.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float u0 = __uint_as_float(ur[j] << 16), u1 = __uint_as_float(ur[j] & 0xffff0000u);
+              pk[j] = pack_bf16x2(__uint_as_float(v[c][2 * j]) * gelu_grad(u0, args.gelu_tanh),
+                                  __uint_as_float(v[c][2 * j + 1]) * gelu_grad(u1, args.gelu_tanh));
+            }
+          } else if (EPI == EPI_DLOGITS) {
+            // dz = (softmax(z) - onehot(target)) / n_scored on scored rows and
+            // valid columns, 0 elsewhere (padding columns included)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float d[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = col0 + 2 * j + e;
+                const float p = ex2_approx(fmaf(__uint_as_float(v[c][2 * j + e]), LOG2E, -d_lse2));
+                d[e] = (d_tgt >= 0 && col < N) ? (p - (col == d_tgt ? 1.f : 0.f)) * d_inv : 0.f;
+              }
+              pk[j] = pack_bf16x2(d[0], d[1]);
+            }
+          } else {
+            uint32_t bc[16];   // bias as bf16 pairs
+            load_bias32_raw(bias_p, col0, N, bc);
+            uint32_t zp[EPI == EPI_GELU_SAVE ? 16 : 1];   // EPI_GELU_SAVE: the pre-activation as bf16 pairs
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float b0 = __uint_as_float(bc[j] << 16), b1 = __uint_as_float(bc[j] & 0xffff0000u);
+              const float x0 = __uint_as_float(v[c][2 * j]), x1 = __uint_as_float(v[c][2 * j + 1]);
+              if (kGelu) {
+                const uint64_t z2 = f2_add(f2_pack(x0, x1), f2_pack(b0, b1));
+                const uint64_t y2 = args.gelu_tanh ? gelu_tanh_x2(z2) : gelu_erf_x2(z2);
+                float a, b;
+                f2_unpack(y2, a, b);
+                pk[j] = pack_bf16x2(a, b);
+                if (EPI == EPI_GELU_SAVE) {
+                  f2_unpack(z2, a, b);
+                  zp[EPI == EPI_GELU_SAVE ? j : 0] = pack_bf16x2(a, b);
+                }
+              } else {
+                pk[j] = pack_bf16x2(x0 + b0, x1 + b1);
+              }
+            }
+            if (EPI == EPI_GELU_SAVE) stage_and_send(zp, &tmD, col0);
+          }
+          stage_and_send(pk, &tmC, col0);
         }
       }
     }
@@ -468,44 +556,65 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
 }
 
 
-// The residual epilogue's 4 KB staging per warp does not fit next to the ring
-// at BN = 256 (gemm_tc_pick_bn never picks it there).
-template <int BN, int EPI>
+// The fp32 epilogues' 4 KB staging per warp does not fit next to the ring at
+// BN = 256 (gemm_tc_pick_bn never picks it there). The backward layouts are
+// instantiated only with the epilogues the backward pass uses.
+template <int BN, int EPI, int LAYOUT>
 constexpr bool tc_supported() {
-  return !(EPI == EPI_RESID && BN == 256);
+  if ((EPI == EPI_RESID || EPI == EPI_F32) && BN == 256) return false;
+  if (LAYOUT == LAYOUT_B_MN) return EPI == EPI_BIAS || EPI == EPI_F32 || EPI == EPI_DGELU;
+  if (LAYOUT == LAYOUT_MN_MN) return EPI == EPI_F32;
+  if (LAYOUT == LAYOUT_A_MN) return false;
+  return EPI != EPI_DGELU && EPI != EPI_F32;
 }
 
-template <int BN, int EPI>
-cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC, const GemmArgs& a,
-                       int num_sms, cudaStream_t s) {
-  if constexpr (!tc_supported<BN, EPI>()) {
+template <int BN, int EPI, int LAYOUT>
+cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC, const CUtensorMap& tD,
+                       const GemmArgs& a, int num_sms, cudaStream_t s) {
+  if constexpr (!tc_supported<BN, EPI, LAYOUT>()) {
     return cudaErrorInvalidValue;
   } else {
     using L = TcLayout<BN, EPI>;
     const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
     const int grid = std::min(tiles, num_sms);
     if (grid <= 0) return cudaSuccess;
-    return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, tA, tB, tC, a);
+    return launch_pdl(gemm_tc_kernel<BN, EPI, LAYOUT>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, tA, tB, tC,
+                      tD, a);
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int LAYOUT>
 cudaError_t set_attr_one() {
-  if constexpr (!tc_supported<BN, EPI>()) return cudaSuccess;
-  else return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if constexpr (!tc_supported<BN, EPI, LAYOUT>()) return cudaSuccess;
+  else return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               TcLayout<BN, EPI>::SMEM_BYTES);
 }
 
-template <int BN>
+template <int BN, int LAYOUT>
 cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
-                      const GemmArgs& a, int num_sms, cudaStream_t s) {
+                      const CUtensorMap& tD, const GemmArgs& a, int num_sms, cudaStream_t s) {
   switch (epi) {
-    case EPI_BIAS: return launch_one<BN, EPI_BIAS>(tA, tB, tC, a, num_sms, s);
-    case EPI_GELU: return launch_one<BN, EPI_GELU>(tA, tB, tC, a, num_sms, s);
-    case EPI_RESID: return launch_one<BN, EPI_RESID>(tA, tB, tC, a, num_sms, s);
+    case EPI_BIAS: return launch_one<BN, EPI_BIAS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_GELU: return launch_one<BN, EPI_GELU, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_RESID: return launch_one<BN, EPI_RESID, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
     case EPI_LMHEAD:
-      return a.out != nullptr ? launch_one<BN, EPI_LMHEAD_LOGITS>(tA, tB, tC, a, num_sms, s)
-                              : launch_one<BN, EPI_LMHEAD>(tA, tB, tC, a, num_sms, s);
+      return a.out != nullptr ? launch_one<BN, EPI_LMHEAD_LOGITS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s)
+                              : launch_one<BN, EPI_LMHEAD, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_F32: return launch_one<BN, EPI_F32, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_DGELU: return launch_one<BN, EPI_DGELU, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_DLOGITS: return launch_one<BN, EPI_DLOGITS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_GELU_SAVE: return launch_one<BN, EPI_GELU_SAVE, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BN>
+cudaError_t launch_layout(int layout, int epi, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
+                          const CUtensorMap& tD, const GemmArgs& a, int num_sms, cudaStream_t s) {
+  switch (layout) {
+    case LAYOUT_KK: return launch_bn<BN, LAYOUT_KK>(epi, tA, tB, tC, tD, a, num_sms, s);
+    case LAYOUT_B_MN: return launch_bn<BN, LAYOUT_B_MN>(epi, tA, tB, tC, tD, a, num_sms, s);
+    case LAYOUT_MN_MN: return launch_bn<BN, LAYOUT_MN_MN>(epi, tA, tB, tC, tD, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -542,8 +651,8 @@ bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t 
 int gemm_tc_n_tiles(int N, int bn) { return (bn / 64) * ((N + bn - 1) / bn); }   // TcLayout::GROUPS per tile
 
 int gemm_tc_pick_bn(int M, int N, int num_sms, int epi) {
-  // The residual epilogue runs with tiles of at most 192 columns.
-  const int max_bn = epi == EPI_RESID ? 192 : 256;
+  // The fp32 epilogues run with tiles of at most 192 columns.
+  const int max_bn = (epi == EPI_RESID || epi == EPI_F32) ? 192 : 256;
   // G2_GEMM_BN=64|128|192|256 pins the tile width (tests use it to cover
   // every instantiation); otherwise the width is chosen by the cost model below.
   if (const char* e = getenv("G2_GEMM_BN")) {
@@ -574,29 +683,47 @@ int gemm_tc_pick_bn(int M, int N, int num_sms, int epi) {
 }
 
 cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
-                           const GemmArgs& a, int num_sms, cudaStream_t s) {
+                           const GemmArgs& a, int num_sms, cudaStream_t s, int layout, const CUtensorMap* tD) {
+  if (epi == EPI_GELU_SAVE && tD == nullptr) return cudaErrorInvalidValue;
+  const CUtensorMap& d = tD ? *tD : tC;
   switch (bn) {
-    case 256: return launch_bn<256>(epi, tA, tB, tC, a, num_sms, s);
-    case 192: return launch_bn<192>(epi, tA, tB, tC, a, num_sms, s);
-    case 128: return launch_bn<128>(epi, tA, tB, tC, a, num_sms, s);
-    case 64: return launch_bn<64>(epi, tA, tB, tC, a, num_sms, s);
+    case 256: return launch_layout<256>(layout, epi, tA, tB, tC, d, a, num_sms, s);
+    case 192: return launch_layout<192>(layout, epi, tA, tB, tC, d, a, num_sms, s);
+    case 128: return launch_layout<128>(layout, epi, tA, tB, tC, d, a, num_sms, s);
+    case 64: return launch_layout<64>(layout, epi, tA, tB, tC, d, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
 
-cudaError_t gemm_tc_set_attributes() {
+namespace {
+template <int BN, int LAYOUT>
+cudaError_t set_attr_layout() {
   cudaError_t e = cudaSuccess;
-#define G2_ATTR(BN)                                              \
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_BIAS>();        \
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU>();        \
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID>();       \
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD>();      \
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD_LOGITS>();
-  G2_ATTR(256)
-  G2_ATTR(192)
-  G2_ATTR(128)
-  G2_ATTR(64)
-#undef G2_ATTR
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_BIAS, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD_LOGITS, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_F32, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_DGELU, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_DLOGITS, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU_SAVE, LAYOUT>();
+  return e;
+}
+template <int BN>
+cudaError_t set_attr_bn() {
+  cudaError_t e = set_attr_layout<BN, LAYOUT_KK>();
+  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_B_MN>();
+  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_MN_MN>();
+  return e;
+}
+}  // namespace
+
+cudaError_t gemm_tc_set_attributes() {
+  cudaError_t e = set_attr_bn<256>();
+  if (e == cudaSuccess) e = set_attr_bn<192>();
+  if (e == cudaSuccess) e = set_attr_bn<128>();
+  if (e == cudaSuccess) e = set_attr_bn<64>();
   return e;
 }
 

@@ -26,31 +26,11 @@
 #include "gpt2.h"
 #include "decode.h"
 #include "kernels.h"
+#include "model.h"
 
 using namespace g2;
 
 namespace {
-
-constexpr int NUM_BN = 4;
-constexpr int BN_CHOICES[NUM_BN] = {256, 192, 128, 64};
-inline int bn_index(int bn) { return bn == 256 ? 0 : (bn == 192 ? 1 : (bn == 128 ? 2 : 3)); }
-
-inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
-
-
-struct LayerPtrs {
-  const void *ln1_g, *ln1_b, *attn_w, *attn_b, *attn_proj_w, *attn_proj_b;
-  const void *ln2_g, *ln2_b, *fc_w, *fc_b, *mlp_proj_w, *mlp_proj_b;
-};
-
-struct WeightMaps {  // one tensor map per candidate tile width
-  CUtensorMap attn[NUM_BN], proj[NUM_BN], fc[NUM_BN], mproj[NUM_BN];
-};
-
-struct Plan {
-  size_t x, h, qkv, y, f, part, tgt, tok, attn, attn_flags, status, total;
-  int attn_pairs;
-};
 
 Plan plan_workspace(const gpt2_config_t& c, int max_B, int max_T) {
   const long M = (long)max_B * max_T;
@@ -116,32 +96,9 @@ int device_setup(int* dev_out, int* sms_out) {
   return GPT2_OK;
 }
 
-bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
 
-struct gpt2_model {
-  gpt2_config_t cfg;
-  bool bf16;
-  int device = 0, num_sms = 0;
-  int max_B = 0, max_T = 0;
-  long max_M = 0;
-  const void *wte = nullptr, *wpe = nullptr, *lnf_g = nullptr, *lnf_b = nullptr;
-  std::vector<LayerPtrs> layers;
-  std::vector<WeightMaps> maps;
-  CUtensorMap wte_map[NUM_BN];
-  uint8_t* ws = nullptr;
-  Plan plan;
-  float* x = nullptr;
-  void *h = nullptr, *qkv = nullptr, *y = nullptr, *f = nullptr;
-  float2* part = nullptr;
-  float* tgt = nullptr;
-  float* tok = nullptr;
-  int* status = nullptr;
-  AttnScratch attn;            // attention work counters (in the zeroed status block), split flags, partials
-  uint64_t launches = 0;
-  cudaEvent_t ev_lm_begin = nullptr, ev_lm_end = nullptr;
-};
 
 namespace {
 

@@ -29,19 +29,36 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // plus the fused lm_head / cross-entropy epilogue.
 // EPI_LMHEAD_LOGITS is the lm_head kernel that also writes the logits;
 // gemm_tc_launch picks it for EPI_LMHEAD when GemmArgs::out is set.
-enum EpiKind : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_LMHEAD = 3, EPI_LMHEAD_LOGITS = 4 };
+// The training pass adds: EPI_GELU_SAVE (EPI_GELU that also stores the
+// pre-activation through tmD), EPI_F32 (fp32 result, TMA store), EPI_DGELU
+// (result times the GELU derivative at a saved pre-activation, bf16) and
+// EPI_DLOGITS (the cross-entropy gradient of the logits, bf16).
+enum EpiKind : int {
+  EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_LMHEAD = 3, EPI_LMHEAD_LOGITS = 4,
+  EPI_F32 = 5, EPI_DGELU = 6, EPI_DLOGITS = 7, EPI_GELU_SAVE = 8
+};
+
+// Operand layouts of the tcgen05 GEMM C = A . B^T (bit set: the operand is
+// stored MN-major, its M or N index contiguous, as the transposed operands of
+// the backward pass are: dX = dY W reads W [N_out, K_in] as B MN-major; dW =
+// dY^T X reads dY [tokens, out] as A MN-major and X [tokens, in] as B MN-major).
+enum GemmLayout : int { LAYOUT_KK = 0, LAYOUT_A_MN = 1, LAYOUT_B_MN = 2, LAYOUT_MN_MN = 3 };
 
 struct GemmArgs {
-  int M, N, K;
-  const void* bias;        // [N] of the operand dtype (NULL for the lm_head)
-  void* out;               // EPI_BIAS/GELU: [M, ldo] operand dtype; EPI_RESID: fp32 [M, ldo] (+=);
-                           // EPI_LMHEAD: fp32 logits [M, ldo] or NULL
+  int M, N, K;             // K need not be a multiple of 64: the tail reads as zero
+  const void* bias;        // [N] of the operand dtype, or NULL (no bias; NULL for the lm_head)
+  void* out;               // EPI_BIAS/GELU/DGELU/DLOGITS: [M, ldo] bf16; EPI_RESID: fp32 [M, ldo] (+=);
+                           // EPI_F32: fp32 [M, ldo]; EPI_LMHEAD: fp32 logits [M, ldo] or NULL
   long long ldo;
-  const int* targets;      // EPI_LMHEAD: [M]
+  const int* targets;      // EPI_LMHEAD, EPI_DLOGITS: [M]
   float2* part;            // EPI_LMHEAD: per (column group, row) (max, sum exp(z - max)), [n_groups, M]
   float* tgt_logit;        // EPI_LMHEAD: [M] logit of the target column
   int* status;
-  int gelu_tanh;           // EPI_GELU: 1 = tanh approximation, 0 = exact erf form
+  int gelu_tanh;           // EPI_GELU(_SAVE), EPI_DGELU: 1 = tanh approximation, 0 = exact erf form
+  const void* aux;         // EPI_DGELU: saved pre-activation u, bf16 [M, ld_aux]
+  long long ld_aux;
+  const float* row_lse;    // EPI_DLOGITS: natural-log log-sum-exp of each row [M]
+  const int* n_scored;     // EPI_DLOGITS: number of rows with a target (device int)
 };
 
 // ---- tensor maps (host) -------------------------------------------------
@@ -67,12 +84,17 @@ constexpr int LMHEAD_MIN_BN = 128;
 inline size_t lmhead_groups_max(int V) { return (size_t)((V + 63) / 64) + 3; }
 
 // ---- tcgen05 GEMM (bf16) -------------------------------------------------
-// C = A[M,K] . B[N,K]^T with the epilogue `epi`. K % 64 == 0, N % 8 == 0.
-// tmA: box 128 x 64 over A; tmB: box BN x 64 over B, BN from gemm_tc_pick_bn;
-// tmC: the output map (make_tmap_out_*; unused by EPI_LMHEAD).
+// C = A[M,K] . B[N,K]^T with the epilogue `epi`. N % 8 == 0.
+// K-major operands: tmA box 128 x 64 over A [M, K], tmB box BN x 64 over
+// B [N, K] (make_tmap_bf16), BN from gemm_tc_pick_bn. MN-major operands
+// (layout bits): the operand is stored [K, M] or [K, N] and read in boxes of
+// 64 x 64 (make_tmap_bf16 with box_rows 64). tmC: the output map
+// (make_tmap_out_*; unused by EPI_LMHEAD); tmD: EPI_GELU_SAVE's
+// pre-activation output (bf16, like tmC).
 int gemm_tc_pick_bn(int M, int N, int num_sms, int epi);
 cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
-                           const GemmArgs& a, int num_sms, cudaStream_t s);
+                           const GemmArgs& a, int num_sms, cudaStream_t s, int layout = LAYOUT_KK,
+                           const CUtensorMap* tmD = nullptr);
 cudaError_t gemm_tc_set_attributes();
 
 // ---- SIMT fp32 GEMM (fp32 mode) ------------------------------------------
@@ -83,7 +105,7 @@ cudaError_t gemm_simt_launch(int epi, const float* A, const float* W, const Gemm
 cudaError_t embed_launch(bool bf16, const int* ids, const void* wte, const void* wpe, float* x, int M, int T,
                          int C, int V, int* status, cudaStream_t s);
 cudaError_t layernorm_launch(bool bf16, const float* x, const void* g, const void* b, void* out, int M, int C,
-                             cudaStream_t s);
+                             cudaStream_t s, float* x_save = nullptr);
 
 // ---- sinusoidal position table (bf16 or fp32 [n_ctx, C]) -------------------
 cudaError_t sinusoidal_wpe_launch(bool bf16, void* wpe, int n_ctx, int C, cudaStream_t s);
@@ -111,15 +133,21 @@ struct AttnScratch {
 };
 // bytes of flags + partials that never limit the split of a (B, T, H) problem
 size_t attention_scratch_bytes(int B, int T, int H);
+// lse_out (training forward; if not NULL): per (b, h, query) the log2 of
+// the softmax normaliser of the scores scaled by log2(e)/sqrt(d_head), [B, H, T];
+// no query tile is split then.
 cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, int C, const AttnScratch* scratch,
-                                int* status, cudaStream_t s);
+                                int* status, cudaStream_t s, float* lse_out = nullptr);
 cudaError_t attention_launch(bool bf16, const void* qkv, void* y, int B, int T, int H, int C,
                              const AttnScratch* scratch, int* status, cudaStream_t s);
 
 // ---- cross-entropy finalisation -------------------------------------------
 // token_loss[m] = logsumexp over column tiles - tgt_logit[m] (0 where the
 // target is negative); loss_out (if not NULL) = mean over scored rows.
+// lse_out (if not NULL) receives each row's log-sum-exp, n_scored_out (if
+// not NULL, with loss_out) the number of scored rows.
 cudaError_t ce_finish_launch(const float2* part, int n_tiles, const float* tgt_logit, const int* targets, int M,
-                             int V, float* token_loss, float* loss_out, int* status, cudaStream_t s);
+                             int V, float* token_loss, float* loss_out, int* status, cudaStream_t s,
+                             float* lse_out = nullptr, int* n_scored_out = nullptr);
 
 }  // namespace g2

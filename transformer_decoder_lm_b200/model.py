@@ -51,6 +51,7 @@ class GPT2Model:
             raise B.GPT2Error(B.ERR_CODE["GPT2_ERR_INVALID_ARG"], "gpt2_workspace_bytes")
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.max_B = max_B
+        self.max_T = max_T
         self.handle, self._keep = B.gpt2_create(self.cfg, weights, self.workspace, max_B, max_T)
 
     @classmethod
@@ -100,6 +101,29 @@ class GPT2Model:
             logits = torch.empty(Bsz, self.vocab, dtype=torch.float32, device=ids_new.device)
         B.gpt2_decode_step(self.handle, kv_cache, ids_new, Bsz, pos, logits, stream)
         return logits
+
+    def new_train_workspace(self) -> torch.Tensor:
+        """The training workspace of gpt2_forward_backward for this handle's max_B x max_T."""
+        n = B.gpt2_train_workspace_bytes(self.cfg, self.max_B, self.max_T)
+        if n == 0:
+            raise B.GPT2Error(B.ERR_CODE["GPT2_ERR_UNSUPPORTED"], "gpt2_train_workspace_bytes")
+        return torch.empty(n, dtype=torch.uint8, device=self.workspace.device)
+
+    def new_grads(self) -> Dict[str, object]:
+        """fp32 gradient buffers shaped like the weights."""
+        def like(t):
+            return torch.empty(t.shape, dtype=torch.float32, device=t.device)
+        w = self.weights
+        return {"wte": like(w["wte"]), "wpe": like(w["wpe"]), "lnf_g": like(w["lnf_g"]), "lnf_b": like(w["lnf_b"]),
+                "layers": [{k: like(lw[k]) for k in B.LAYER_KEYS} for lw in w["layers"]]}
+
+    def forward_backward(self, ids, targets, grads, train_ws, loss_out=None, stream=None):
+        """Loss and the gradient of every weight (gpt2_forward_backward)."""
+        Bsz, T = ids.shape
+        if loss_out is None:
+            loss_out = torch.empty(1, dtype=torch.float32, device=ids.device)
+        B.gpt2_forward_backward(self.handle, ids, targets, Bsz, T, loss_out, grads, train_ws, stream)
+        return loss_out
 
     def status(self, stream=None) -> int:
         return B.gpt2_status(self.handle, stream)
