@@ -79,6 +79,70 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// The embedding sum of embed_kernel and the first block's ln_1 on the row it
+// just formed (bf16, C <= 128 MAXV): x = wte[id] + wpe[t] (fp32, written),
+// h = LayerNorm(x; g, b) with layernorm_kernel's arithmetic.
+template <int MAXV>
+__global__ void __launch_bounds__(256) embed_ln_kernel(const int* __restrict__ ids, const bf16* __restrict__ wte,
+                                                       const bf16* __restrict__ wpe, float* __restrict__ x,
+                                                       const bf16* __restrict__ g, const bf16* __restrict__ b,
+                                                       bf16* __restrict__ h, int M, int Tlen, int C, int V,
+                                                       int* status) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  if (row >= M) {
+    pdl_trigger();
+    return;
+  }
+  int id = ids[row];
+  if (id < 0 || id >= V) {
+    if (lane == 0) record_error(status, DEV_BAD_TOKEN);
+    id = 0;
+  }
+  const bf16* te = wte + (size_t)id * C;
+  const bf16* pe = wpe + (size_t)(row % Tlen) * C;
+  float* xr = x + (size_t)row * C;
+  float4 v[MAXV];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) {
+      const float4 a = Vec4<bf16>::load(te + c), p = Vec4<bf16>::load(pe + c);
+      v[i] = make_float4(a.x + p.x, a.y + p.y, a.z + p.z, a.w + p.w);
+      Vec4<float>::store(xr + c, v[i]);
+      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    }
+  }
+  const float mean = warp_sum(s) / (float)C;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) {
+      const float a = v[i].x - mean, bb = v[i].y - mean, cc = v[i].z - mean, d = v[i].w - mean;
+      q += (a * a + bb * bb) + (cc * cc + d * d);
+    }
+  }
+  const float rstd = rsqrtf(warp_sum(q) / (float)C + 1e-5f);
+  bf16* orow = h + (size_t)row * C;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = (lane + 32 * i) * 4;
+    if (c < C) {
+      const float4 ga = Vec4<bf16>::load(g + c), be = Vec4<bf16>::load(b + c);
+      float4 o;
+      o.x = (v[i].x - mean) * rstd * ga.x + be.x;
+      o.y = (v[i].y - mean) * rstd * ga.y + be.y;
+      o.z = (v[i].z - mean) * rstd * ga.z + be.z;
+      o.w = (v[i].w - mean) * rstd * ga.w + be.w;
+      Vec4<bf16>::store(orow + c, o);
+    }
+  }
+  pdl_trigger();
+}
+
 // C <= 32 lanes * 4 * MAXV = 2048.
 // x_save (training forward): if not NULL, also receives a copy of x, the
 // LayerNorm input the backward pass differentiates at.
@@ -163,6 +227,21 @@ cudaError_t embed_launch(bool bf16_, const int* ids, const void* wte, const void
     embed_kernel<float><<<grid, threads, 0, s>>>(ids, static_cast<const float*>(wte),
                                                   static_cast<const float*>(wpe), x, M, T, C, V, status);
   return cudaGetLastError();
+}
+
+cudaError_t embed_ln_launch(const int* ids, const void* wte, const void* wpe, float* x, const void* g,
+                            const void* b, void* h, int M, int T, int C, int V, int* status, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (C > 2048 || (C & 3)) return cudaErrorInvalidValue;
+  const int threads = 256, grid = (M + 7) / 8;
+  const bf16 *te = static_cast<const bf16*>(wte), *pe = static_cast<const bf16*>(wpe);
+  const bf16 *gp = static_cast<const bf16*>(g), *bp = static_cast<const bf16*>(b);
+  bf16* hp = static_cast<bf16*>(h);
+  if (C <= 768) return launch_pdl(embed_ln_kernel<6>, grid, threads, 0, s, ids, te, pe, x, gp, bp, hp, M, T, C, V, status);
+  if (C <= 1024) return launch_pdl(embed_ln_kernel<8>, grid, threads, 0, s, ids, te, pe, x, gp, bp, hp, M, T, C, V, status);
+  if (C <= 1280) return launch_pdl(embed_ln_kernel<10>, grid, threads, 0, s, ids, te, pe, x, gp, bp, hp, M, T, C, V, status);
+  if (C <= 1664) return launch_pdl(embed_ln_kernel<13>, grid, threads, 0, s, ids, te, pe, x, gp, bp, hp, M, T, C, V, status);
+  return launch_pdl(embed_ln_kernel<16>, grid, threads, 0, s, ids, te, pe, x, gp, bp, hp, M, T, C, V, status);
 }
 
 cudaError_t layernorm_launch(bool bf16_, const float* x, const void* g, const void* b, void* out, int M, int C,

@@ -54,6 +54,7 @@ Plan plan_workspace(const gpt2_config_t& c, int max_B, int max_T) {
   p.attn_flags = o; o += align256((size_t)p.attn_pairs * ATTN_PAIR_FLAGS * 4);
   p.attn = o;   o += align256((size_t)p.attn_pairs * ATTN_PART_FLOATS * 4);
   p.status = o; o += 256;
+  p.ln_cnt = o; o += align256((size_t)((M + 127) / 128) * 4);
   p.total = o;
   return p;
 }
@@ -103,9 +104,15 @@ int device_setup(int* dev_out, int* sms_out) {
 namespace {
 
 // One Linear layer of the schedule.
+// ln_g / ln_b (EPI_RESID_LN): the LayerNorm that follows, its output into m->h.
 int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, const void* W, const CUtensorMap* wmaps,
-               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s) {
+               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s,
+               const void* ln_g = nullptr, const void* ln_b = nullptr) {
   GemmArgs a{};
+  a.ln_g = ln_g;
+  a.ln_b = ln_b;
+  a.ln_out = m->h;
+  a.row_counter = m->ln_cnt;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -162,12 +169,28 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     if (rc != GPT2_OK) return rc;    \
   } while (0)
 
-  G2_CK(embed_launch(m->bf16, ids, m->wte, m->wpe, m->x, M, T, C, V, m->status, s));
+  // bf16 on the tensor cores: every LayerNorm rides on the kernel before it
+  // (the embedding, or the residual GEMM through EPI_RESID_LN); otherwise
+  // each is a launch of its own
+  const bool fused_ln = m->bf16 && M > GEMV_MAX_M;
+  if (fused_ln) {
+    const LayerPtrs& L0 = m->layers[0];
+    G2_CK(embed_ln_launch(ids, m->wte, m->wpe, m->x, L0.ln1_g, L0.ln1_b, m->h, M, T, C, V, m->status, s));
+  } else {
+    G2_CK(embed_launch(m->bf16, ids, m->wte, m->wpe, m->x, M, T, C, V, m->status, s));
+  }
   m->launches += 1;
   for (int l = 0; l < c.n_layer; ++l) {
     const LayerPtrs& L = m->layers[l];
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
-    G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
+    const bool last = l + 1 == c.n_layer;
+    // the LayerNorm after this block: the next block's ln_1, or ln_f
+    const void* next_g = last ? m->lnf_g : m->layers[l + 1].ln1_g;
+    const void* next_b = last ? m->lnf_b : m->layers[l + 1].ln1_b;
+    if (!fused_ln) {
+      G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
+      m->launches += 1;
+    }
     G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C, m->qkv, 3 * C, s));
     if (kv_cache) {   // k and v of positions 0..T-1 of every sequence into this layer's cache
       const size_t es = m->bf16 ? 2 : 4;
@@ -178,14 +201,26 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
                                 2 * C * es, T, cudaMemcpyDeviceToDevice, s));
     }
     G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, &m->attn, m->status, s));
-    G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
-    G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
+    if (fused_ln) {
+      G2_RC(run_linear(m, EPI_RESID_LN, m->y, &tm_y, L.attn_proj_w, W->proj, &out_x, L.attn_proj_b, M, C, C, m->x, C, s,
+                       L.ln2_g, L.ln2_b));
+    } else {
+      G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
+      G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
+      m->launches += 1;
+    }
     G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, &out_f, L.fc_b, M, 4 * C, C, m->f, 4 * C, s));
-    G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C, s));
-    m->launches += 7;
+    if (fused_ln)
+      G2_RC(run_linear(m, EPI_RESID_LN, m->f, &tm_f, L.mlp_proj_w, W->mproj, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C,
+                       s, next_g, next_b));
+    else
+      G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C, s));
+    m->launches += 5;
   }
-  G2_CK(layernorm_launch(m->bf16, m->x, m->lnf_g, m->lnf_b, m->h, M, C, s));
-  m->launches += 1;
+  if (!fused_ln) {
+    G2_CK(layernorm_launch(m->bf16, m->x, m->lnf_g, m->lnf_b, m->h, M, C, s));
+    m->launches += 1;
+  }
 
   if (logits || targets) {
     GemmArgs a{};
@@ -378,6 +413,7 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
   m->tgt = reinterpret_cast<float*>(ws + p.tgt);
   m->tok = reinterpret_cast<float*>(ws + p.tok);
   m->status = reinterpret_cast<int*>(ws + p.status);
+  m->ln_cnt = reinterpret_cast<int*>(ws + p.ln_cnt);
   m->attn.sched = reinterpret_cast<unsigned*>(ws + p.status + 64);
   m->attn.flags = reinterpret_cast<int*>(ws + p.attn_flags);
   m->attn.part = reinterpret_cast<float*>(ws + p.attn);
@@ -403,6 +439,7 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
     }
   }
   if (cudaMemset(m->status, 0, 256) != cudaSuccess ||
+      cudaMemset(m->ln_cnt, 0, (size_t)((maxM + 127) / 128) * 4) != cudaSuccess ||
       (p.attn_pairs && cudaMemset(m->attn.flags, 0, (size_t)p.attn_pairs * ATTN_PAIR_FLAGS * 4) != cudaSuccess) ||
       cudaDeviceSynchronize() != cudaSuccess) {
     delete m;
@@ -457,6 +494,9 @@ int gpt2_status(gpt2_handle_t h, void* stream) {
   int bits = 0;
   if (cudaMemcpy(&bits, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
   if (bits && cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return GPT2_ERR_CUDA;
+  // a kernel that gave up may have left the fused LayerNorm's arrival counters mid-count
+  if ((bits & DEV_TIMEOUT) && cudaMemset(h->ln_cnt, 0, (size_t)((h->max_M + 127) / 128) * 4) != cudaSuccess)
+    return GPT2_ERR_CUDA;
   if (bits & DEV_TIMEOUT) return GPT2_ERR_DEVICE_TIMEOUT;
   if (bits & DEV_BAD_TOKEN) return GPT2_ERR_BAD_TOKEN;
   if (bits & DEV_NO_TARGETS) return GPT2_ERR_NO_TARGETS;
