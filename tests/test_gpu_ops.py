@@ -295,3 +295,63 @@ def test_fill_sinusoidal_wpe(G, n_ctx, C):
     assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 * 1.0001)
     with pytest.raises(G.GPT2Error):
         G.gpt2_fill_sinusoidal_wpe(G.GPT2_FP32, f32, n_ctx, C + 1)   # odd C
+
+
+@pytest.mark.parametrize("C", [768, 1024, 1600])
+def test_embed_layernorm_fused(G, C):
+    """The embedding sum and ln_1 in one kernel: x as gpt2_op_embed writes it,
+    h = LayerNorm(x) against the oracle (one bf16 rounding)."""
+    M, T, V = 3 * 77, 77, 999
+    rng = np.random.default_rng(C + 1)
+    ids = rng.integers(0, V, size=M).astype(np.int32)
+    wte, wpe = bf16_exact(rng, (V, C), 0.5), bf16_exact(rng, (T, C), 0.5)
+    g, b = bf16_exact(rng, (C,), 1.0), bf16_exact(rng, (C,), 0.2)
+    x = torch.empty(M, C, dtype=torch.float32, device="cuda")
+    h = torch.empty(M, C, dtype=torch.bfloat16, device="cuda")
+    st = status_word()
+    G.gpt2_op_embed_layernorm(torch.from_numpy(ids).cuda(), dev(wte, "bf16"), dev(wpe, "bf16"), M, T, C, V,
+                              dev(g, "bf16"), dev(b, "bf16"), x, h, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rx = wte[ids].astype(np.float64) + wpe[np.arange(M) % T]
+    assert max_abs(x.cpu().numpy(), rx) <= 1e-6
+    rh = O.layer_norm(rx, g.astype(np.float64), b.astype(np.float64))
+    got = h.float().cpu().numpy()
+    assert np.all(np.abs(got - rh) <= np.abs(rh) * 2.0 ** -8 + 1e-4)
+
+
+@pytest.mark.parametrize("shape", [(4096, 768, 768), (4096, 768, 3072), (1000, 1024, 1024), (300, 1600, 6400),
+                                   (130, 64, 128)])
+def test_linear_resid_layernorm_fused(G, shape):
+    """x += A W^T + b and h = LayerNorm(x) in one kernel (the last CTA of each
+    128-row block normalises it): x against the oracle's sum, h against the
+    oracle's LayerNorm of the exact sum, twice in a row (the arrival
+    counters are left zeroed), and h bit-identical to the separate
+    LayerNorm kernel run on the same x."""
+    M, N, K = shape
+    rng = np.random.default_rng(M + N + K)
+    A = bf16_exact(rng, (M, K))
+    W = bf16_exact(rng, (N, K), 1.0 / math.sqrt(K))
+    bias = bf16_exact(rng, (N,), 0.1)
+    g, b = bf16_exact(rng, (N,), 1.0), bf16_exact(rng, (N,), 0.2)
+    x0 = rng.standard_normal((M, N)).astype(np.float32)
+    counters = torch.zeros((M + 127) // 128, dtype=torch.int32, device="cuda")
+    st = status_word()
+    d = [dev(A, "bf16"), dev(W, "bf16"), dev(bias, "bf16")]
+    for rep in range(2):
+        x = dev(x0, "fp32")
+        h = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        G.gpt2_op_linear_resid_ln(d[0], d[1], d[2], M, N, K, x, dev(g, "bf16"), dev(b, "bf16"), h, counters, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert int(counters.abs().sum().item()) == 0
+        rx = x0 + O.linear(A.astype(np.float64), W.astype(np.float64), bias.astype(np.float64))
+        gx = x.cpu().numpy()
+        assert max_abs(gx, rx) <= 1e-4 * max(1.0, math.sqrt(K) / 16)
+        rh = O.layer_norm(gx.astype(np.float64), g.astype(np.float64), b.astype(np.float64))
+        got = h.float().cpu().numpy()
+        assert np.all(np.abs(got - rh) <= np.abs(rh) * 2.0 ** -8 + 1e-4)
+        h2 = torch.empty_like(h)
+        G.gpt2_op_layernorm(G.GPT2_BF16, x, dev(g, "bf16"), dev(b, "bf16"), M, N, h2)
+        torch.cuda.synchronize()
+        assert torch.equal(h, h2)

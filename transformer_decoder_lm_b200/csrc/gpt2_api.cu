@@ -590,6 +590,47 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
   return gemm_tc_launch(epilogue, bn, ta, tb, tc, a, sms, s) == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
+int gpt2_op_embed_layernorm(const int32_t* ids, const void* wte, const void* wpe, int M, int T, int C, int V,
+                            const void* g, const void* b, float* x, void* h, int* status, void* stream) {
+  if (!ids || !aligned16(wte) || !aligned16(wpe) || !aligned16(g) || !aligned16(b) || !aligned16(x) || !aligned16(h) ||
+      M < 0 || T < 1 || C < 64 || (C % 64) || C > 2048 || V < 1)
+    return GPT2_ERR_INVALID_ARG;
+  return embed_ln_launch(ids, wte, wpe, x, g, b, h, M, T, C, V, status, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? GPT2_OK
+             : GPT2_ERR_CUDA;
+}
+
+int gpt2_op_linear_resid_ln(const void* A, const void* W, const void* bias, int M, int N, int K, float* x,
+                            const void* g, const void* b, void* h, int* counters, int* status, void* stream) {
+  if (!aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(x) || !aligned16(g) || !aligned16(b) ||
+      !aligned16(h) || !counters || M < 1 || N < 64 || (N % 64) || N > 2048 || K < 64 || (K % 64))
+    return GPT2_ERR_INVALID_ARG;
+  int sms = 0;
+  int rc = device_setup(nullptr, &sms);
+  if (rc != GPT2_OK) return rc;
+  const int bn = gemm_tc_pick_bn(M, N, sms, EPI_RESID_LN);
+  CUtensorMap ta, tb, tc;
+  if (!make_tmap_bf16(&ta, A, M, K, K, 128) || !make_tmap_bf16(&tb, W, N, K, K, bn) ||
+      !make_tmap_out_f32(&tc, x, M, N, N))
+    return GPT2_ERR_CUDA;
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.bias = bias;
+  a.out = x;
+  a.ldo = N;
+  a.status = status;
+  a.ln_g = g;
+  a.ln_b = b;
+  a.ln_out = h;
+  a.row_counter = counters;
+  return gemm_tc_launch(EPI_RESID_LN, bn, ta, tb, tc, a, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? GPT2_OK
+             : GPT2_ERR_CUDA;
+}
+
 int gpt2_fill_sinusoidal_wpe(int dtype, void* wpe, int n_ctx, int C, void* stream) {
   if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || !wpe || n_ctx < 1 || C < 2 || (C % 2)) return GPT2_ERR_INVALID_ARG;
   return sinusoidal_wpe_launch(dtype == GPT2_BF16, wpe, n_ctx, C, static_cast<cudaStream_t>(stream)) == cudaSuccess
