@@ -404,15 +404,6 @@ def run_kernel(args):
         qkv, y = rnd(M, 3 * C), torch.empty(M, C, dtype=bf, device="cuda")
         fn = lambda: G.gpt2_op_attention(G.GPT2_BF16, qkv, WL.batch, WL.seq, H, C, y)
         flops = WL.batch * 2.0 * C * WL.seq * (WL.seq + 1)
-    elif k in ("attn_proj_ln", "mlp_proj_ln"):
-        N, K = (C, C) if k == "attn_proj_ln" else (C, 4 * C)
-        A, W, b = rnd(M, K), rnd(N, K, scale=0.02), rnd(N, scale=0.01)
-        g, be = rnd(N), rnd(N)
-        x = torch.zeros(M, N, dtype=torch.float32, device="cuda")
-        h = torch.empty(M, N, dtype=bf, device="cuda")
-        counters = torch.zeros((M + 127) // 128, dtype=torch.int32, device="cuda")
-        fn = lambda: G.gpt2_op_linear_resid_ln(A, W, b, M, N, K, x, g, be, h, counters)
-        flops = 2.0 * M * N * K
     elif k == "embed_ln":
         ids = torch.from_numpy(rng.integers(0, V, size=M).astype(np.int32)).cuda()
         wte, wpe = rnd(V, C, scale=0.02), rnd(WL.n_ctx, C, scale=0.02)
@@ -488,7 +479,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None,
                     help="run one step alone: lmhead, lmhead_ce (no logits), c_attn, attn_proj, c_fc, mlp_proj, "
-                         "attn_proj_ln, mlp_proj_ln (with the fused LayerNorm), attention, embed, embed_ln, layernorm, "
+                         "attention, embed, embed_ln (with the first ln_1), layernorm, "
                          "decode (one key/value-cache decoding step, B 4, context 1024)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

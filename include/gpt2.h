@@ -196,22 +196,15 @@ enum { GPT2_EPI_BIAS = 0, GPT2_EPI_BIAS_GELU = 1, GPT2_EPI_BIAS_RESID = 2, GPT2_
 int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const void* bias,
                    int M, int N, int K, void* out, int* status, void* stream);
 
-/* The two fused steps of the bf16 forward pass (M > 16), where each
- * LayerNorm rides on the kernel before it ("Hand-writing GPT-2 from scratch:
- * the Transformer decoder core modules in PyTorch", section 3.2: the Pre-LN
- * block's residual add followed by the next sub-layer's LayerNorm):
- *   gpt2_op_embed_layernorm:  x fp32 [M, C] = wte[ids] + wpe[m % T] and
- *                             h bf16 [M, C] = LayerNorm(x; g, b)
- *   gpt2_op_linear_resid_ln:  x fp32 [M, N] += A W^T + bias, then
- *                             h bf16 [M, N] = LayerNorm(x; g, b)
- * bf16 weights, C or N a multiple of 64 and <= 2048, K a multiple of 64.
- * `counters` (gpt2_op_linear_resid_ln): ceil(M / 128) int32 of device memory
- * that the caller zeroes once; every call leaves them zeroed again. Calls
- * sharing counters must not overlap on the GPU. */
+/* The bf16 forward pass (M > 16) computes the embedding sum and the first
+ * block's ln_1 in one kernel ("Hand-writing GPT-2 from scratch: the
+ * Transformer decoder core modules in PyTorch", section 4.1 step 1 then the
+ * Pre-LN block of section 3.2): x fp32 [M, C] = wte[ids] + wpe[m % T] as
+ * gpt2_op_embed writes it, and h bf16 [M, C] = LayerNorm(x; g, b). bf16
+ * tables and g, b; C a multiple of 64 and <= 2048. Ids outside [0, V) read
+ * row 0 and set GPT2_ERR_BAD_TOKEN in *status. */
 int gpt2_op_embed_layernorm(const int32_t* ids, const void* wte, const void* wpe, int M, int T, int C, int V,
                             const void* g, const void* b, float* x, void* h, int* status, void* stream);
-int gpt2_op_linear_resid_ln(const void* A, const void* W, const void* bias, int M, int N, int K, float* x,
-                            const void* g, const void* b, void* h, int* counters, int* status, void* stream);
 
 /* ---- incremental decoding with a key/value cache ---------------------------
  * The pages' generate loops feed the sequence back one new token at a time

@@ -13,7 +13,7 @@ from .binding import (  # noqa: F401
     gpt2_kv_cache_bytes, gpt2_prefill, gpt2_decode_step,
     gpt2_workspace_bytes, gpt2_create, gpt2_forward, gpt2_loss, gpt2_forward_loss, gpt2_status,
     gpt2_error_string, gpt2_destroy, gpt2_launch_count, gpt2_set_timing_events, GPT2_TIMED_LMHEAD,
-    gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear, gpt2_op_embed_layernorm, gpt2_op_linear_resid_ln,
+    gpt2_op_embed, gpt2_op_layernorm, gpt2_op_linear, gpt2_op_embed_layernorm,
     gpt2_op_attention, gpt2_op_lmhead_ce_workspace_bytes, gpt2_op_lmhead_ce, make_config,
     gpt2_op_lmhead_ce_noalloc, GPT2_NOALLOC_SCRATCH_BYTES,
     gpt2_train_workspace_bytes, gpt2_forward_backward, gpt2_op_linear_dgrad, gpt2_op_linear_wgrad,

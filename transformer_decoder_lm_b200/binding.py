@@ -86,7 +86,6 @@ def _load():
         "gpt2_op_attention": (i, [i, vp, i, i, i, i, vp, vp, vp]),
         "gpt2_fill_sinusoidal_wpe": (i, [i, vp, i, i, vp]),
         "gpt2_op_embed_layernorm": (i, [vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, vp]),
-        "gpt2_op_linear_resid_ln": (i, [vp, vp, vp, i, i, i, vp, vp, vp, vp, vp, vp, vp]),
         "gpt2_op_lmhead_ce_workspace_bytes": (sz, [i, i, i]),
         "gpt2_op_lmhead_ce": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
         "gpt2_op_lmhead_ce_noalloc": (i, [i, vp, vp, vp, i, i, i, vp, vp, vp, vp, vp]),
@@ -241,11 +240,6 @@ def gpt2_op_linear(dtype, epilogue, A, W, bias, M, N, K, out, status=None, strea
 def gpt2_op_embed_layernorm(ids, wte, wpe, M, T, C, V, g, b, x, h, status=None, stream=None):
     _check(lib.gpt2_op_embed_layernorm(_ptr(ids), _ptr(wte), _ptr(wpe), M, T, C, V, _ptr(g), _ptr(b), _ptr(x), _ptr(h),
                                        _ptr(status), _stream(stream)), "gpt2_op_embed_layernorm")
-
-
-def gpt2_op_linear_resid_ln(A, W, bias, M, N, K, x, g, b, h, counters, status=None, stream=None):
-    _check(lib.gpt2_op_linear_resid_ln(_ptr(A), _ptr(W), _ptr(bias), M, N, K, _ptr(x), _ptr(g), _ptr(b), _ptr(h),
-                                       _ptr(counters), _ptr(status), _stream(stream)), "gpt2_op_linear_resid_ln")
 
 
 def gpt2_fill_sinusoidal_wpe(dtype, wpe, n_ctx, C, stream=None):

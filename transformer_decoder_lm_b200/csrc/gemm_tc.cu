@@ -50,7 +50,6 @@
 namespace g2 {
 
 constexpr int TC_BM = 128;
-constexpr int TC_BM_LN = TC_BM;
 constexpr int TC_BK = 64;
 constexpr int TC_STAGES = 4;
 template <int BN, int EPI>
@@ -64,7 +63,7 @@ struct TcLayout {
   static constexpr int THREADS = 32 * (2 + EPI_WARPS);
   // per epilogue warp: one 32 x 32 chunk (bf16: 2 KB, fp32 residual: 4 KB),
   // or 8 logits rows x 64 fp32 (2 KB)
-  static constexpr bool F32_OUT = EPI == EPI_RESID || EPI == EPI_RESID_LN || EPI == EPI_F32;
+  static constexpr bool F32_OUT = EPI == EPI_RESID || EPI == EPI_F32;
   static constexpr int STAGE_BUF_BYTES = F32_OUT ? 4096 : 2048;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
@@ -95,66 +94,23 @@ __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int 
   }
 }
 
-// LayerNorm of rows m0 + first, m0 + first + stride, ... (< M, < m0 + 128)
-// of the fp32 residual stream x [M, C] into out bf16 [M, C], one warp per
-// row, the row in registers (C <= 128 MAXV): the arithmetic of
-// layernorm_kernel (mean, then the centred second moment, eps 1e-5 inside
-// the square root). x is read through L2 (other SMs wrote it).
-template <int MAXV>
-__device__ __noinline__ void ln_rows(const float* __restrict__ x, const bf16* __restrict__ g,
-                                     const bf16* __restrict__ b, bf16* __restrict__ out, int m0, int M, int C,
-                                     int first, int stride, int lane) {
-  for (int r = first; r < TC_BM_LN; r += stride) {
-    const int row = m0 + r;
-    if (row >= M) break;
-    const float* xr = x + (size_t)row * C;
-    float4 v[MAXV];
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int c = (lane + 32 * i) * 4;
-      if (c < C) v[i] = __ldcg(reinterpret_cast<const float4*>(xr + c));
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i)
-      if ((lane + 32 * i) * 4 < C) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float mean = s / (float)C;
-    float q = 0.f;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i)
-      if ((lane + 32 * i) * 4 < C) {
-        const float a = v[i].x - mean, bb = v[i].y - mean, cc = v[i].z - mean, d = v[i].w - mean;
-        q += (a * a + bb * bb) + (cc * cc + d * d);
-      }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-    const float rstd = rsqrtf(q / (float)C + 1e-5f);
-    bf16* orow = out + (size_t)row * C;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int c = (lane + 32 * i) * 4;
-      if (c < C) {
-        const uint2 gu = __ldg(reinterpret_cast<const uint2*>(g + c));
-        const uint2 bu = __ldg(reinterpret_cast<const uint2*>(b + c));
-        const float o0 = (v[i].x - mean) * rstd * __uint_as_float(gu.x << 16) + __uint_as_float(bu.x << 16);
-        const float o1 = (v[i].y - mean) * rstd * __uint_as_float(gu.x & 0xffff0000u) + __uint_as_float(bu.x & 0xffff0000u);
-        const float o2 = (v[i].z - mean) * rstd * __uint_as_float(gu.y << 16) + __uint_as_float(bu.y << 16);
-        const float o3 = (v[i].w - mean) * rstd * __uint_as_float(gu.y & 0xffff0000u) + __uint_as_float(bu.y & 0xffff0000u);
-        *reinterpret_cast<uint2*>(orow + c) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
-      }
-    }
+// Tile t's (row block, column block). Row blocks are taken in groups of
+// `group` (<= 0: all of them): within a group the row block varies fastest,
+// so the CTAs working at the same time share column tiles of B; groups run
+// one after the other, so those CTAs also write neighbouring column tiles of
+// the same rows of the output.
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int group, int& m_blk, int& n_blk) {
+  if (group <= 0 || group >= m_tiles) {
+    m_blk = t % m_tiles;
+    n_blk = t / m_tiles;
+    return;
   }
-}
-
-__device__ __forceinline__ void ln_rows_any(const float* x, const bf16* g, const bf16* b, bf16* out, int m0, int M,
-                                            int C, int first, int stride, int lane) {
-  if (C <= 768) ln_rows<6>(x, g, b, out, m0, M, C, first, stride, lane);
-  else if (C <= 1024) ln_rows<8>(x, g, b, out, m0, M, C, first, stride, lane);
-  else if (C <= 1280) ln_rows<10>(x, g, b, out, m0, M, C, first, stride, lane);
-  else if (C <= 1664) ln_rows<13>(x, g, b, out, m0, M, C, first, stride, lane);
-  else ln_rows<16>(x, g, b, out, m0, M, C, first, stride, lane);
+  const int per_group = group * n_tiles;
+  const int g = t / per_group;
+  const int r = t - g * per_group;
+  const int rows = min(group, m_tiles - g * group);   // the last group may be short
+  m_blk = g * group + r % rows;
+  n_blk = r / rows;
 }
 
 // Derivative of the GELU at the pre-activation u: exact form
@@ -178,7 +134,6 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   constexpr bool kLM = EPI == EPI_LMHEAD || EPI == EPI_LMHEAD_LOGITS;
   constexpr bool kAmn = (LAYOUT & LAYOUT_A_MN) != 0, kBmn = (LAYOUT & LAYOUT_B_MN) != 0;
   constexpr bool kGelu = EPI == EPI_GELU || EPI == EPI_GELU_SAVE;
-  constexpr bool kResid = EPI == EPI_RESID || EPI == EPI_RESID_LN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
@@ -188,7 +143,6 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* ln_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);   // EPI_RESID_LN
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -235,8 +189,10 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
       uint32_t issued = 0, issued_parity = 0;   // per stage: a load was issued / its barrier phase parity
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % m_tiles) * TC_BM;
-        const int n0 = (tile / m_tiles) * BN;
+        int m_blk, n_blk;
+        tile_coords(tile, m_tiles, n_tiles, args.m_group, m_blk, n_blk);
+        const int m0 = m_blk * TC_BM;
+        const int n0 = n_blk * BN;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -337,7 +293,8 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      int m_blk, n_blk;
+      tile_coords(tile, m_tiles, n_tiles, args.m_group, m_blk, n_blk);
       const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
       const int row0 = m0 + q * 32;          // first row of this warp
       const int row = row0 + lane;
@@ -497,7 +454,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (kResid)
+            if (EPI == EPI_RESID)
               tma_reduce_add_2d(map, sbuf, col0, row0);
             else
               tma_store_2d(map, sbuf, col0, row0);
@@ -577,32 +534,6 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           }
           stage_and_send(pk, &tmC, col0);
         }
-        if (EPI == EPI_RESID_LN) {
-          // The tile's sums have landed in x once its reduce-adds complete;
-          // count the tile for its 128-row block, and the epilogue warps of
-          // the CTA that completes a block normalise the block's rows. No
-          // CTA ever waits on another: the last arrival does the work.
-          if (lane == 0) {
-            bulk_wait_all();
-            fence_proxy_async_global();
-          }
-          __syncwarp();
-          store_pending = false;
-          named_barrier_sync(1, L::EPI_WARPS * 32);
-          if (warp == 2 && lane == 0) {
-            __threadfence();
-            *ln_flag = atomicAdd(args.row_counter + m_blk, 1) == n_tiles - 1;
-          }
-          named_barrier_sync(1, L::EPI_WARPS * 32);
-          if (*ln_flag) {
-            __threadfence();
-            fence_proxy_async_global();
-            ln_rows_any(static_cast<const float*>(args.out), static_cast<const bf16*>(args.ln_g),
-                        static_cast<const bf16*>(args.ln_b), static_cast<bf16*>(args.ln_out), m0, M, N, warp - 2,
-                        L::EPI_WARPS, lane);
-            if (warp == 2 && lane == 0) args.row_counter[m_blk] = 0;   // every tile of the block has arrived
-          }
-        }
       }
     }
     if (!kLM && lane == 0) bulk_wait_all();
@@ -652,8 +583,7 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
 // instantiated only with the epilogues the backward pass uses.
 template <int BN, int EPI, int LAYOUT>
 constexpr bool tc_supported() {
-  if ((EPI == EPI_RESID || EPI == EPI_RESID_LN || EPI == EPI_F32) && BN == 256) return false;
-  if (EPI == EPI_RESID_LN) return LAYOUT == LAYOUT_KK;
+  if ((EPI == EPI_RESID || EPI == EPI_F32) && BN == 256) return false;
   if (LAYOUT == LAYOUT_B_MN) return EPI == EPI_BIAS || EPI == EPI_F32 || EPI == EPI_DGELU;
   if (LAYOUT == LAYOUT_MN_MN) return EPI == EPI_F32;
   if (LAYOUT == LAYOUT_A_MN) return false;
@@ -696,7 +626,6 @@ cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, con
     case EPI_DGELU: return launch_one<BN, EPI_DGELU, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
     case EPI_DLOGITS: return launch_one<BN, EPI_DLOGITS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
     case EPI_GELU_SAVE: return launch_one<BN, EPI_GELU_SAVE, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_RESID_LN: return launch_one<BN, EPI_RESID_LN, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -745,7 +674,7 @@ int gemm_tc_n_tiles(int N, int bn) { return (bn / 64) * ((N + bn - 1) / bn); }  
 
 int gemm_tc_pick_bn(int M, int N, int num_sms, int epi) {
   // The fp32 epilogues run with tiles of at most 192 columns.
-  const int max_bn = (epi == EPI_RESID || epi == EPI_RESID_LN || epi == EPI_F32) ? 192 : 256;
+  const int max_bn = (epi == EPI_RESID || epi == EPI_F32) ? 192 : 256;
   // G2_GEMM_BN=64|128|192|256 pins the tile width (tests use it to cover
   // every instantiation); otherwise the width is chosen by the cost model below.
   if (const char* e = getenv("G2_GEMM_BN")) {
@@ -801,7 +730,6 @@ cudaError_t set_attr_layout() {
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_DGELU, LAYOUT>();
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_DLOGITS, LAYOUT>();
   if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU_SAVE, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID_LN, LAYOUT>();
   return e;
 }
 template <int BN>

@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -54,7 +55,6 @@ Plan plan_workspace(const gpt2_config_t& c, int max_B, int max_T) {
   p.attn_flags = o; o += align256((size_t)p.attn_pairs * ATTN_PAIR_FLAGS * 4);
   p.attn = o;   o += align256((size_t)p.attn_pairs * ATTN_PART_FLOATS * 4);
   p.status = o; o += 256;
-  p.ln_cnt = o; o += align256((size_t)((M + 127) / 128) * 4);
   p.total = o;
   return p;
 }
@@ -78,6 +78,14 @@ struct DeviceInfo {
 };
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
+
+// Row blocks per tile group of the lm_head GEMM (see tile_coords in
+// gemm_tc.cu); G2_LMHEAD_GROUP overrides the default (for measurements).
+int lmhead_group(bool with_logits) {
+  if (const char* e = getenv("G2_LMHEAD_GROUP")) return atoi(e);
+  (void)with_logits;
+  return 0;
+}
 
 int device_setup(int* dev_out, int* sms_out) {
   int dev = 0;
@@ -104,15 +112,9 @@ int device_setup(int* dev_out, int* sms_out) {
 namespace {
 
 // One Linear layer of the schedule.
-// ln_g / ln_b (EPI_RESID_LN): the LayerNorm that follows, its output into m->h.
 int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, const void* W, const CUtensorMap* wmaps,
-               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s,
-               const void* ln_g = nullptr, const void* ln_b = nullptr) {
+               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s) {
   GemmArgs a{};
-  a.ln_g = ln_g;
-  a.ln_b = ln_b;
-  a.ln_out = m->h;
-  a.row_counter = m->ln_cnt;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -169,9 +171,8 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     if (rc != GPT2_OK) return rc;    \
   } while (0)
 
-  // bf16 on the tensor cores: every LayerNorm rides on the kernel before it
-  // (the embedding, or the residual GEMM through EPI_RESID_LN); otherwise
-  // each is a launch of its own
+  // bf16 on the tensor cores: the first block's ln_1 rides on the embedding
+  // kernel; every other LayerNorm is a launch of its own
   const bool fused_ln = m->bf16 && M > GEMV_MAX_M;
   if (fused_ln) {
     const LayerPtrs& L0 = m->layers[0];
@@ -183,11 +184,7 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
   for (int l = 0; l < c.n_layer; ++l) {
     const LayerPtrs& L = m->layers[l];
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
-    const bool last = l + 1 == c.n_layer;
-    // the LayerNorm after this block: the next block's ln_1, or ln_f
-    const void* next_g = last ? m->lnf_g : m->layers[l + 1].ln1_g;
-    const void* next_b = last ? m->lnf_b : m->layers[l + 1].ln1_b;
-    if (!fused_ln) {
+    if (l > 0 || !fused_ln) {
       G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
       m->launches += 1;
     }
@@ -201,26 +198,14 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
                                 2 * C * es, T, cudaMemcpyDeviceToDevice, s));
     }
     G2_CK(attention_launch(m->bf16, m->qkv, m->y, B, T, H, C, &m->attn, m->status, s));
-    if (fused_ln) {
-      G2_RC(run_linear(m, EPI_RESID_LN, m->y, &tm_y, L.attn_proj_w, W->proj, &out_x, L.attn_proj_b, M, C, C, m->x, C, s,
-                       L.ln2_g, L.ln2_b));
-    } else {
-      G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
-      G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
-      m->launches += 1;
-    }
+    G2_RC(run_linear(m, EPI_RESID, m->y, &tm_y, L.attn_proj_w, W ? W->proj : nullptr, &out_x, L.attn_proj_b, M, C, C, m->x, C, s));
+    G2_CK(layernorm_launch(m->bf16, m->x, L.ln2_g, L.ln2_b, m->h, M, C, s));
     G2_RC(run_linear(m, EPI_GELU, m->h, &tm_h, L.fc_w, W ? W->fc : nullptr, &out_f, L.fc_b, M, 4 * C, C, m->f, 4 * C, s));
-    if (fused_ln)
-      G2_RC(run_linear(m, EPI_RESID_LN, m->f, &tm_f, L.mlp_proj_w, W->mproj, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C,
-                       s, next_g, next_b));
-    else
-      G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C, s));
-    m->launches += 5;
+    G2_RC(run_linear(m, EPI_RESID, m->f, &tm_f, L.mlp_proj_w, W ? W->mproj : nullptr, &out_x, L.mlp_proj_b, M, C, 4 * C, m->x, C, s));
+    m->launches += 6;
   }
-  if (!fused_ln) {
-    G2_CK(layernorm_launch(m->bf16, m->x, m->lnf_g, m->lnf_b, m->h, M, C, s));
-    m->launches += 1;
-  }
+  G2_CK(layernorm_launch(m->bf16, m->x, m->lnf_g, m->lnf_b, m->h, M, C, s));
+  m->launches += 1;
 
   if (logits || targets) {
     GemmArgs a{};
@@ -234,6 +219,7 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     a.part = m->part;
     a.tgt_logit = m->tgt;
     a.status = m->status;
+    a.m_group = lmhead_group(logits != nullptr);
     int n_tiles;
     if (m->ev_lm_begin) G2_CK(cudaEventRecord(m->ev_lm_begin, s));
     if (m->bf16) {
@@ -413,7 +399,6 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
   m->tgt = reinterpret_cast<float*>(ws + p.tgt);
   m->tok = reinterpret_cast<float*>(ws + p.tok);
   m->status = reinterpret_cast<int*>(ws + p.status);
-  m->ln_cnt = reinterpret_cast<int*>(ws + p.ln_cnt);
   m->attn.sched = reinterpret_cast<unsigned*>(ws + p.status + 64);
   m->attn.flags = reinterpret_cast<int*>(ws + p.attn_flags);
   m->attn.part = reinterpret_cast<float*>(ws + p.attn);
@@ -439,7 +424,6 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
     }
   }
   if (cudaMemset(m->status, 0, 256) != cudaSuccess ||
-      cudaMemset(m->ln_cnt, 0, (size_t)((maxM + 127) / 128) * 4) != cudaSuccess ||
       (p.attn_pairs && cudaMemset(m->attn.flags, 0, (size_t)p.attn_pairs * ATTN_PAIR_FLAGS * 4) != cudaSuccess) ||
       cudaDeviceSynchronize() != cudaSuccess) {
     delete m;
@@ -494,9 +478,6 @@ int gpt2_status(gpt2_handle_t h, void* stream) {
   int bits = 0;
   if (cudaMemcpy(&bits, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
   if (bits && cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return GPT2_ERR_CUDA;
-  // a kernel that gave up may have left the fused LayerNorm's arrival counters mid-count
-  if ((bits & DEV_TIMEOUT) && cudaMemset(h->ln_cnt, 0, (size_t)((h->max_M + 127) / 128) * 4) != cudaSuccess)
-    return GPT2_ERR_CUDA;
   if (bits & DEV_TIMEOUT) return GPT2_ERR_DEVICE_TIMEOUT;
   if (bits & DEV_BAD_TOKEN) return GPT2_ERR_BAD_TOKEN;
   if (bits & DEV_NO_TARGETS) return GPT2_ERR_NO_TARGETS;
@@ -601,36 +582,6 @@ int gpt2_op_embed_layernorm(const int32_t* ids, const void* wte, const void* wpe
              : GPT2_ERR_CUDA;
 }
 
-int gpt2_op_linear_resid_ln(const void* A, const void* W, const void* bias, int M, int N, int K, float* x,
-                            const void* g, const void* b, void* h, int* counters, int* status, void* stream) {
-  if (!aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(x) || !aligned16(g) || !aligned16(b) ||
-      !aligned16(h) || !counters || M < 1 || N < 64 || (N % 64) || N > 2048 || K < 64 || (K % 64))
-    return GPT2_ERR_INVALID_ARG;
-  int sms = 0;
-  int rc = device_setup(nullptr, &sms);
-  if (rc != GPT2_OK) return rc;
-  const int bn = gemm_tc_pick_bn(M, N, sms, EPI_RESID_LN);
-  CUtensorMap ta, tb, tc;
-  if (!make_tmap_bf16(&ta, A, M, K, K, 128) || !make_tmap_bf16(&tb, W, N, K, K, bn) ||
-      !make_tmap_out_f32(&tc, x, M, N, N))
-    return GPT2_ERR_CUDA;
-  GemmArgs a{};
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.bias = bias;
-  a.out = x;
-  a.ldo = N;
-  a.status = status;
-  a.ln_g = g;
-  a.ln_b = b;
-  a.ln_out = h;
-  a.row_counter = counters;
-  return gemm_tc_launch(EPI_RESID_LN, bn, ta, tb, tc, a, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? GPT2_OK
-             : GPT2_ERR_CUDA;
-}
-
 int gpt2_fill_sinusoidal_wpe(int dtype, void* wpe, int n_ctx, int C, void* stream) {
   if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || !wpe || n_ctx < 1 || C < 2 || (C % 2)) return GPT2_ERR_INVALID_ARG;
   return sinusoidal_wpe_launch(dtype == GPT2_BF16, wpe, n_ctx, C, static_cast<cudaStream_t>(stream)) == cudaSuccess
@@ -678,6 +629,7 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
   a.part = part;
   a.tgt_logit = tgt;
   a.status = status;
+  a.m_group = lmhead_group(logits_or_null != nullptr);
   int n_tiles;
   if (dtype == GPT2_BF16) {
     if (C % 64) return GPT2_ERR_UNSUPPORTED;

@@ -33,13 +33,9 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // pre-activation through tmD), EPI_F32 (fp32 result, TMA store), EPI_DGELU
 // (result times the GELU derivative at a saved pre-activation, bf16) and
 // EPI_DLOGITS (the cross-entropy gradient of the logits, bf16).
-// EPI_RESID_LN is EPI_RESID followed by the next LayerNorm of the schedule:
-// the CTA that completes the last tile of a 128-row block (a per-block
-// arrival counter) normalises those rows of the updated residual stream and
-// writes them (bf16) to ln_out, so no separate LayerNorm launch is needed.
 enum EpiKind : int {
   EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_LMHEAD = 3, EPI_LMHEAD_LOGITS = 4,
-  EPI_F32 = 5, EPI_DGELU = 6, EPI_DLOGITS = 7, EPI_GELU_SAVE = 8, EPI_RESID_LN = 9
+  EPI_F32 = 5, EPI_DGELU = 6, EPI_DLOGITS = 7, EPI_GELU_SAVE = 8
 };
 
 // Operand layouts of the tcgen05 GEMM C = A . B^T (bit set: the operand is
@@ -63,10 +59,7 @@ struct GemmArgs {
   long long ld_aux;
   const float* row_lse;    // EPI_DLOGITS: natural-log log-sum-exp of each row [M]
   const int* n_scored;     // EPI_DLOGITS: number of rows with a target (device int)
-  const void* ln_g;        // EPI_RESID_LN: gamma, beta bf16 [N] of the LayerNorm that follows
-  const void* ln_b;
-  void* ln_out;            // EPI_RESID_LN: its output, bf16 [M, N]
-  int* row_counter;        // EPI_RESID_LN: one zeroed int per 128-row block (left zeroed)
+  int m_group;             // tile order: row blocks per group (0 = all: row block fastest over the whole M)
 };
 
 // ---- tensor maps (host) -------------------------------------------------

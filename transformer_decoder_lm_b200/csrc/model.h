@@ -31,7 +31,7 @@ struct WeightMaps {  // one tensor map per candidate tile width
 
 // Byte offsets of the workspace slices (gpt2_create).
 struct Plan {
-  size_t x, h, qkv, y, f, part, tgt, tok, attn, attn_flags, status, ln_cnt, total;
+  size_t x, h, qkv, y, f, part, tgt, tok, attn, attn_flags, status, total;
   int attn_pairs;
 };
 
@@ -55,7 +55,6 @@ struct gpt2_model {
   float* tgt = nullptr;
   float* tok = nullptr;
   int* status = nullptr;
-  int* ln_cnt = nullptr;       // per 128-row block arrival counters of the fused LayerNorm (zeroed)
   g2::AttnScratch attn;        // attention work counters (in the zeroed status block), split flags, partials
   uint64_t launches = 0;
   cudaEvent_t ev_lm_begin = nullptr, ev_lm_end = nullptr;
