@@ -48,6 +48,7 @@
 // Every wait is bounded (common.cuh); on a timeout the CTA records
 // GPT2_ERR_DEVICE_TIMEOUT, drains its copies and MMAs, frees TMEM and exits.
 #include <math.h>
+#include <stdlib.h>
 
 #include <utility>
 
@@ -78,11 +79,11 @@ constexpr int AT_SMEM = OFF_BAR + NUM_BARS * 8 + 16;   // + TMEM holder, abort f
 constexpr uint32_t TMEM_COLS = 256;   // S: cols [0,128) fp32, O: [128,192) fp32, P: [192,256) bf16 pairs
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 192;
 constexpr float RESCALE_THRESHOLD = 8.0f;                // log2 units
-// Bit k set: pair k of every 8 takes 2^x by ex2_poly_x2 on the FMA pipe
-// instead of the SFU. Measured at d_head 64 the SFU is not the limit (the
-// softmax is issue- and latency-bound), so the polynomial only adds
-// instructions: all exponentials stay on the SFU.
-constexpr uint32_t POLY_PAIRS = 0x00u;
+// Exponential split (template argument kPoly of the kernel): bit k set, pair
+// k of every 8 takes 2^x by ex2_poly_x2 on the FMA pipe instead of the SFU.
+// G2_ATTN_POLY = 0, 2, 3 or 4 (pairs of every 8 on the FMA pipe) selects an
+// instantiation for measurements; the default keeps all on the SFU.
+constexpr uint32_t POLY_MASKS[5] = {0x00u, 0x00u, 0x11u, 0x49u, 0x55u};
 constexpr int AT_MAX_CLS = 64;
 enum : uint32_t { ROLE_WHOLE = 0, ROLE_FIRST = 1, ROLE_SECOND = 2 };
 constexpr int PART_M = 128 * 64, PART_L = PART_M + 128;  // partial: O as [16][128 rows][4], then m[128], l[128]
@@ -151,7 +152,7 @@ __device__ __forceinline__ bool wait_flag(const int* f, volatile int* abort_flag
 // whole SMs drain. sched[0] counts the items handed out past the grid, sched[1] counts finished CTAs;
 // the last CTA to finish sets both back to 0 for the next launch.
 // kSplit: the plan splits some query tiles (the merge code is compiled in).
-template <bool kSplit>
+template <bool kSplit, uint32_t kPoly>
 __global__ void __launch_bounds__(AT_THREADS, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_y, int B,
                        int T, int H, int C, float scale_log2, const __grid_constant__ AttnPlan plan,
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         }
         l *= alpha;
         // x = s log2(e)/sqrt(D) - m, p = 2^x: pairs of columns in packed fp32;
-        // POLY_PAIRS of every 8 pairs take 2^x on the FMA pipe, the rest on the SFU
+        // the kPoly pairs of every 8 take 2^x on the FMA pipe, the rest on the SFU
         const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m, -m);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[4][16];
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
           for (int e = 0; e < 16; ++e) {
             const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sc2, nm2);
             float p0, p1;
-            if ((POLY_PAIRS >> (e & 7)) & 1u) {
+            if ((kPoly >> (e & 7)) & 1u) {
               ex2_poly_x2(x, p0, p1);
             } else {
               float x0, x1;
@@ -656,6 +657,7 @@ AttnPlan make_plan(int BH, int QT, int slots, int cap_pairs, int* n_split) {
   // more than twice a slot's average share: splitting costs a second Q load
   // and the merge, and only pays where a few long items set the kernel's length
   long target = 2 * ((tiles + slots - 1) / slots);
+  if (const char* e = getenv("G2_ATTN_SPLIT")) target = atol(e) > 0 ? atol(e) : target;   // measurements
   if (target < 2) target = 2;
   int split_of[AT_MAX_CLS / 2];
   int S = 0;
@@ -695,6 +697,16 @@ AttnPlan make_plan(int BH, int QT, int slots, int cap_pairs, int* n_split) {
 }
 }  // namespace
 
+template <bool kSplit>
+auto pick_kernel(int poly) {
+  switch (poly) {
+    case 2: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[2]>;
+    case 3: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[3]>;
+    case 4: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[4]>;
+  }
+  return attn_fwd_tc_kernel<kSplit, POLY_MASKS[0]>;
+}
+
 size_t attention_scratch_bytes(int B, int T, int H) {
   const size_t QT = ((size_t)T + AT_BQ - 1) / AT_BQ;
   return QT * (size_t)B * H * (ATTN_PART_FLOATS * 4 + ATTN_PAIR_FLAGS * 4);
@@ -710,17 +722,23 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  int poly = 0;
+  if (const char* pe = getenv("G2_ATTN_POLY")) poly = atoi(pe);
+  if (poly < 0 || poly > 4) poly = 0;
+  const auto kfalse = pick_kernel<false>(poly);
+  const auto ktrue = pick_kernel<true>(poly);
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_fwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
-    // two CTAs share an SM only with the largest shared-memory carveout
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_fwd_tc_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_fwd_tc_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               cudaSharedmemCarveoutMaxShared);
+    cudaError_t e = cudaSuccess;
+    for (int pk = 0; pk < 5 && e == cudaSuccess; ++pk) {
+      void (*ks[2])(CUtensorMap, CUtensorMap, int, int, int, int, float, AttnPlan, unsigned*, int*, float*, int, int*,
+                    float*) = {pick_kernel<false>(pk), pick_kernel<true>(pk)};
+      for (auto k : ks) {
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+        // two CTAs share an SM only with the largest shared-memory carveout
+        if (e == cudaSuccess)
+          e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+      }
+    }
     int sms = 0;
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) slots[dev] = 2 * sms;   // __launch_bounds__(AT_THREADS, 2)
@@ -729,12 +747,15 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
     if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&own[dev].part), g_attn_part);
     // the register split must fit in what the launch allocates, or the
     // softmax warps' setmaxnreg.inc would never be granted
-    cudaFuncAttributes fa[2];
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[0], attn_fwd_tc_kernel<false>);
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[1], attn_fwd_tc_kernel<true>);
+    for (int pk = 0; pk < 5 && e == cudaSuccess; ++pk) {
+      cudaFuncAttributes fa[2];
+      e = cudaFuncGetAttributes(&fa[0], pick_kernel<false>(pk));
+      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[1], pick_kernel<true>(pk));
+      if (e != cudaSuccess) return e;
+      for (const cudaFuncAttributes& f : fa)
+        if (f.numRegs * AT_THREADS < 128 * (REG_SOFTMAX + REG_OTHER)) return cudaErrorInvalidConfiguration;
+    }
     if (e != cudaSuccess) return e;
-    for (const cudaFuncAttributes& f : fa)
-      if (f.numRegs * AT_THREADS < 128 * (REG_SOFTMAX + REG_OTHER)) return cudaErrorInvalidConfiguration;
     own[dev].cap_pairs = OWN_PAIRS;
     attr_set[dev] = true;
   }
@@ -754,9 +775,9 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
   const int grid = items < slots[dev] ? items : slots[dev];
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)AT_D));
   if (n_split)
-    return launch_pdl(attn_fwd_tc_kernel<true>, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
+    return launch_pdl(ktrue, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
                       plan, sc.sched, sc.flags, sc.part, n_split * BH * ATTN_PAIR_FLAGS, status, lse_out);
-  return launch_pdl(attn_fwd_tc_kernel<false>, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
+  return launch_pdl(kfalse, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, ty, B, T, H, C, scale_log2,
                     plan, sc.sched, sc.flags, sc.part, 0, status, lse_out);
 }
 

@@ -94,25 +94,6 @@ __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int 
   }
 }
 
-// Tile t's (row block, column block). Row blocks are taken in groups of
-// `group` (<= 0: all of them): within a group the row block varies fastest,
-// so the CTAs working at the same time share column tiles of B; groups run
-// one after the other, so those CTAs also write neighbouring column tiles of
-// the same rows of the output.
-__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int group, int& m_blk, int& n_blk) {
-  if (group <= 0 || group >= m_tiles) {
-    m_blk = t % m_tiles;
-    n_blk = t / m_tiles;
-    return;
-  }
-  const int per_group = group * n_tiles;
-  const int g = t / per_group;
-  const int r = t - g * per_group;
-  const int rows = min(group, m_tiles - g * group);   // the last group may be short
-  m_blk = g * group + r % rows;
-  n_blk = r / rows;
-}
-
 // Derivative of the GELU at the pre-activation u: exact form
 // d/du [u Phi(u)] = Phi(u) + u phi(u); tanh form
 // d/du [u (1 + tanh(k (u + c u^3))) / 2] = (1 + t) / 2 + u (1 - t^2) k (1 + 3 c u^2) / 2.
@@ -189,10 +170,8 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
       uint32_t issued = 0, issued_parity = 0;   // per stage: a load was issued / its barrier phase parity
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int m_blk, n_blk;
-        tile_coords(tile, m_tiles, n_tiles, args.m_group, m_blk, n_blk);
-        const int m0 = m_blk * TC_BM;
-        const int n0 = n_blk * BN;
+        const int m0 = (tile % m_tiles) * TC_BM;
+        const int n0 = (tile / m_tiles) * BN;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -293,8 +272,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      int m_blk, n_blk;
-      tile_coords(tile, m_tiles, n_tiles, args.m_group, m_blk, n_blk);
+      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
       const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
       const int row0 = m0 + q * 32;          // first row of this warp
       const int row = row0 + lane;

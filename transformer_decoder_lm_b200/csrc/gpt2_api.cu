@@ -79,14 +79,6 @@ struct DeviceInfo {
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
 
-// Row blocks per tile group of the lm_head GEMM (see tile_coords in
-// gemm_tc.cu); G2_LMHEAD_GROUP overrides the default (for measurements).
-int lmhead_group(bool with_logits) {
-  if (const char* e = getenv("G2_LMHEAD_GROUP")) return atoi(e);
-  (void)with_logits;
-  return 0;
-}
-
 int device_setup(int* dev_out, int* sms_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPT2_ERR_CUDA;
@@ -219,7 +211,6 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     a.part = m->part;
     a.tgt_logit = m->tgt;
     a.status = m->status;
-    a.m_group = lmhead_group(logits != nullptr);
     int n_tiles;
     if (m->ev_lm_begin) G2_CK(cudaEventRecord(m->ev_lm_begin, s));
     if (m->bf16) {
@@ -629,7 +620,6 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
   a.part = part;
   a.tgt_logit = tgt;
   a.status = status;
-  a.m_group = lmhead_group(logits_or_null != nullptr);
   int n_tiles;
   if (dtype == GPT2_BF16) {
     if (C % 64) return GPT2_ERR_UNSUPPORTED;

@@ -59,7 +59,6 @@ struct GemmArgs {
   long long ld_aux;
   const float* row_lse;    // EPI_DLOGITS: natural-log log-sum-exp of each row [M]
   const int* n_scored;     // EPI_DLOGITS: number of rows with a target (device int)
-  int m_group;             // tile order: row blocks per group (0 = all: row block fastest over the whole M)
 };
 
 // ---- tensor maps (host) -------------------------------------------------
