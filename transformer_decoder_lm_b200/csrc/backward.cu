@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(32 * LNB_WARPS) layernorm_bwd_kernel(
   float* sg = lnb_smem + (size_t)warp * C;
   float* sbt = lnb_smem + (size_t)(LNB_WARPS + warp) * C;
   pdl_wait();
+  pdl_trigger();
   for (int c = lane; c < C; c += 32) {
     sg[c] = 0.f;
     sbt[c] = 0.f;
@@ -162,7 +163,6 @@ __global__ void __launch_bounds__(32 * LNB_WARPS) layernorm_bwd_kernel(
     part_g[(size_t)blockIdx.x * C + c] = a;
     part_b[(size_t)blockIdx.x * C + c] = b;
   }
-  pdl_trigger();
 }
 
 constexpr int COL_ROWS = 128;
@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(256) col_partials_kernel(const T* __restrict__
                                                            float* __restrict__ part) {
   const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   pdl_wait();
+  pdl_trigger();
   if (c0 < N) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const int r0 = blockIdx.y * COL_ROWS, r1 = min(M, r0 + COL_ROWS);
@@ -203,7 +204,6 @@ __global__ void __launch_bounds__(256) col_partials_kernel(const T* __restrict__
 #pragma unroll
     for (int j = 0; j < 8; ++j) part[(size_t)blockIdx.y * N + c0 + j] = acc[j];
   }
-  pdl_trigger();
 }
 
 // out[c] = sum over p of part[p, c], p in order.
@@ -211,12 +211,12 @@ __global__ void __launch_bounds__(256) col_reduce_kernel(const float* __restrict
                                                          float* __restrict__ out) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   pdl_wait();
+  pdl_trigger();
   if (c < N) {
     float s = 0.f;
     for (int p = 0; p < P; ++p) s += part[(size_t)p * N + c];
     out[c] = s;
   }
-  pdl_trigger();
 }
 
 // Dv[(b H + h) T + i] = sum over the head's 64 columns of dO * O: one warp per
@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const bf16* __restri
                                                             float* __restrict__ Dv, int B, int T, int H, int C) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   pdl_wait();
+  pdl_trigger();
   if (row < B * T) {
     const int b = row / T, i = row % T;
     for (int c0 = lane * 8; c0 < C; c0 += 256) {
@@ -242,7 +243,6 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const bf16* __restri
       if ((lane & 7) == 0) Dv[((size_t)b * H + c0 / 64) * T + i] = s;
     }
   }
-  pdl_trigger();
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
   const int g = lane >> 2, t = lane & 3;
   constexpr int CH = AB_D / 8;
   pdl_wait();
+  pdl_trigger();
 
   for (int i = tid; i < AB_T * CH; i += 128) {
     const int r = i / CH, c = (i % CH) * 8;
@@ -441,7 +442,6 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
       *reinterpret_cast<uint32_t*>(ob + (size_t)key1 * ld + 2 * C + col) = pack_bf16x2(dv[dn][2], dv[dn][3]);
     }
   }
-  pdl_trigger();
 }
 
 // dqkv[:, 0:C] = bf16(dq_acc * scale); 8 columns per thread.
@@ -449,6 +449,7 @@ __global__ void __launch_bounds__(256) dq_finish_kernel(const float* __restrict_
                                                         int M, int C, float scale) {
   const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   pdl_wait();
+  pdl_trigger();
   if (i < (long long)M * C) {
     const long long row = i / C, col = i % C;
     const float4 a = *reinterpret_cast<const float4*>(dq_acc + i);
@@ -460,7 +461,6 @@ __global__ void __launch_bounds__(256) dq_finish_kernel(const float* __restrict_
     u.w = pack_bf16x2(c.z * scale, c.w * scale);
     *reinterpret_cast<uint4*>(dqkv + row * 3 * C + col) = u;
   }
-  pdl_trigger();
 }
 
 // dwte[ids[m]] += dx[m]: one warp per row, fp32 atomics (ids checked by the forward).
@@ -468,12 +468,12 @@ __global__ void __launch_bounds__(256) embed_bwd_wte_kernel(const int* __restric
                                                             float* __restrict__ dwte, int M, int C, int V) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   pdl_wait();
+  pdl_trigger();
   if (row < M) {
     const int id = ids[row];
     if (id >= 0 && id < V)
       for (int c = lane; c < C; c += 32) atomicAdd(dwte + (size_t)id * C + c, dx[(size_t)row * C + c]);
   }
-  pdl_trigger();
 }
 
 // dwpe[t, c] = sum over b of dx[b, t, c] for t < T, 0 for T <= t < n_ctx.
@@ -481,6 +481,7 @@ __global__ void __launch_bounds__(256) embed_bwd_wpe_kernel(const float* __restr
                                                             int B, int T, int n_ctx, int C) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   pdl_wait();
+  pdl_trigger();
   if (i < (long long)n_ctx * C) {
     const int t = (int)(i / C), c = (int)(i % C);
     float s = 0.f;
@@ -488,7 +489,6 @@ __global__ void __launch_bounds__(256) embed_bwd_wpe_kernel(const float* __restr
       for (int b = 0; b < B; ++b) s += dx[((size_t)b * T + t) * C + c];
     dwpe[i] = s;
   }
-  pdl_trigger();
 }
 
 }  // namespace

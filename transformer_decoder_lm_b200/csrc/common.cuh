@@ -46,8 +46,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // serialisation: a kernel may start (set up barriers, allocate TMEM, prefetch
 // descriptors) while its predecessor drains, and waits in pdl_wait() until
 // the predecessor has completed and its writes are visible before it reads
-// any of them. Each CTA calls pdl_trigger() once its last output is issued so
-// that the successor can be scheduled. Both are no-ops for plain launches.
+// or writes any global memory. Each CTA calls pdl_trigger() right after its
+// own pdl_wait(), so the successor's CTAs are placed on SMs as soon as they
+// free up and have their set-up done when this kernel completes (every CTA
+// of this kernel is resident by then: the successor launches only once all
+// of them have triggered). Both are no-ops for plain launches.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
@@ -253,6 +256,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 lanes x 16 columns of 32-bit words to TMEM.
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 
 // Instruction descriptor of tcgen05.mma kind::f16 with a K-major A, an
 // MN-major B (B stored with N contiguous), bf16 inputs, fp32 D.

@@ -52,10 +52,8 @@ __global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids,
   const int row = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   pdl_wait();
-  if (row >= M) {
-    pdl_trigger();
-    return;
-  }
+  pdl_trigger();
+  if (row >= M) return;
   int id = ids[row];
   if (id < 0 || id >= V) {
     if (lane == 0) record_error(status, DEV_BAD_TOKEN);
@@ -70,7 +68,6 @@ __global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids,
     const float4 b = Vec4<T>::load(pe + c);
     Vec4<float>::store(xr + c, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
   }
-  pdl_trigger();
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -91,10 +88,8 @@ __global__ void __launch_bounds__(256) embed_ln_kernel(const int* __restrict__ i
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   pdl_wait();
-  if (row >= M) {
-    pdl_trigger();
-    return;
-  }
+  pdl_trigger();
+  if (row >= M) return;
   int id = ids[row];
   if (id < 0 || id >= V) {
     if (lane == 0) record_error(status, DEV_BAD_TOKEN);
@@ -140,7 +135,6 @@ __global__ void __launch_bounds__(256) embed_ln_kernel(const int* __restrict__ i
       Vec4<bf16>::store(orow + c, o);
     }
   }
-  pdl_trigger();
 }
 
 // C <= 32 lanes * 4 * MAXV = 2048.
@@ -154,10 +148,8 @@ __global__ void __launch_bounds__(128) layernorm_kernel(const float* __restrict_
   const int row = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   pdl_wait();
-  if (row >= M) {
-    pdl_trigger();
-    return;
-  }
+  pdl_trigger();
+  if (row >= M) return;
   const float* xr = x + (size_t)row * C;
   // x, gamma and beta are all requested before any of them is used, so a row
   // costs one memory round trip.
@@ -212,7 +204,6 @@ __global__ void __launch_bounds__(128) layernorm_kernel(const float* __restrict_
       Vec4<T>::store(orow + c, o);
     }
   }
-  pdl_trigger();
 }
 
 cudaError_t embed_launch(bool bf16_, const int* ids, const void* wte, const void* wpe, float* x, int M, int T,

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   pdl_wait();   // the operands and the residual stream come from the previous kernel
+  if (threadIdx.x == 0) pdl_trigger();   // the next kernel may start its set-up as SMs free up
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -519,7 +520,6 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   }
 
   __syncthreads();
-  if (threadIdx.x == 0) pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::TMEM_COLS);

@@ -26,6 +26,7 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_bf16_kernel(const bf16* 
                                                                     int N, int K, long long ldo, int gelu_tanh) {
   const int n = blockIdx.x * GEMV_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   pdl_wait();
+  pdl_trigger();
   if (n < N) {
     float acc[GEMV_MAX_M];
 #pragma unroll
@@ -71,7 +72,6 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_bf16_kernel(const bf16* 
       }
     }
   }
-  pdl_trigger();
 }
 }  // namespace
 
