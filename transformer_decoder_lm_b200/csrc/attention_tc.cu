@@ -48,7 +48,6 @@
 // Every wait is bounded (common.cuh); on a timeout the CTA records
 // GPT2_ERR_DEVICE_TIMEOUT, drains its copies and MMAs, frees TMEM and exits.
 #include <math.h>
-#include <stdlib.h>
 
 #include <utility>
 
@@ -79,11 +78,6 @@ constexpr int AT_SMEM = OFF_BAR + NUM_BARS * 8 + 16;   // + TMEM holder, abort f
 constexpr uint32_t TMEM_COLS = 256;   // S: cols [0,128) fp32, O: [128,192) fp32, P: [192,256) bf16 pairs
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 192;
 constexpr float RESCALE_THRESHOLD = 8.0f;                // log2 units
-// Exponential split (template argument kPoly of the kernel): bit k set, pair
-// k of every 8 takes 2^x by ex2_poly_x2 on the FMA pipe instead of the SFU.
-// G2_ATTN_POLY = 0, 2, 3 or 4 (pairs of every 8 on the FMA pipe) selects an
-// instantiation for measurements; the default keeps all on the SFU.
-constexpr uint32_t POLY_MASKS[5] = {0x00u, 0x00u, 0x11u, 0x49u, 0x55u};
 constexpr int AT_MAX_CLS = 64;
 enum : uint32_t { ROLE_WHOLE = 0, ROLE_FIRST = 1, ROLE_SECOND = 2 };
 constexpr int PART_M = 128 * 64, PART_L = PART_M + 128;  // partial: O as [16][128 rows][4], then m[128], l[128]
@@ -152,11 +146,7 @@ __device__ __forceinline__ bool wait_flag(const int* f, volatile int* abort_flag
 // whole SMs drain. sched[0] counts the items handed out past the grid, sched[1] counts finished CTAs;
 // the last CTA to finish sets both back to 0 for the next launch.
 // kSplit: the plan splits some query tiles (the merge code is compiled in).
-// kStream: the softmax waits for the previous P.V first, then turns each
-// 32-key chunk of the S row into P and stores it to TMEM straight away (the
-// exponentials of a chunk never wait on the others' registers); otherwise all
-// 128 probabilities are formed first and stored together.
-template <bool kSplit, uint32_t kPoly, bool kStream>
+template <bool kSplit>
 __global__ void __launch_bounds__(AT_THREADS, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_y, int B,
                        int T, int H, int C, float scale_log2, const __grid_constant__ AttnPlan plan,
@@ -417,69 +407,10 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
           m = m_new;
         }
         l *= alpha;
-        // x = s log2(e)/sqrt(D) - m, p = 2^x: pairs of columns in packed fp32;
-        // the kPoly pairs of every 8 take 2^x on the FMA pipe, the rest on the SFU
+        // x = s log2(e)/sqrt(D) - m, p = 2^x: pairs of columns in packed fp32,
+        // exponentials on the SFU
         const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m, -m);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
-        if (kStream) {
-          if (gj > 0) {   // PV of the previous tile done: the P buffer is free (and O stable)
-            if (!mbar_wait(pv_done, (gj - 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          // chunk c: keys 32c..32c+31 -> 16 packed columns of P at tP + 16c
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pc[16];
-            if (diag && c > qd) {   // keys of this chunk all lie after every row of this warp
-#pragma unroll
-              for (int e = 0; e < 16; ++e) pc[e] = 0u;
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const uint64_t x =
-                    f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sc2, nm2);
-                float p0, p1;
-                if ((kPoly >> (e & 7)) & 1u) {
-                  ex2_poly_x2(x, p0, p1);
-                } else {
-                  float x0, x1;
-                  f2_unpack(x, x0, x1);
-                  p0 = ex2_approx(x0);
-                  p1 = ex2_approx(x1);
-                }
-                ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(p0, p1));
-                pc[e] = pack_bf16x2(p0, p1);
-              }
-            }
-            tmem_st_32x32b_x16(tP + 16 * c, pc);
-          }
-          {
-            const uint64_t s2 = f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3]));
-            float s0, s1;
-            f2_unpack(s2, s0, s1);
-            l += s0 + s1;
-          }
-          // a raised max: O scaled down before this tile's P.V adds to it
-          if (gj > 0 && jj > 0 && __any_sync(0xffffffffu, raise)) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              uint32_t o[32];
-              tmem_ld_32x32b_x32(tO + c * 32, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st_32x32b_x32(tO + c * 32, o);
-            }
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(p_full);
-          continue;
-        }
         uint32_t pk[4][16];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -491,15 +422,9 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sc2, nm2);
-            float p0, p1;
-            if ((kPoly >> (e & 7)) & 1u) {
-              ex2_poly_x2(x, p0, p1);
-            } else {
-              float x0, x1;
-              f2_unpack(x, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(p0, p1));
             pk[c][e] = pack_bf16x2(p0, p1);
           }
@@ -720,7 +645,6 @@ AttnPlan make_plan(int BH, int QT, int slots, int cap_pairs, int* n_split) {
   // more than twice a slot's average share: splitting costs a second Q load
   // and the merge, and only pays where a few long items set the kernel's length
   long target = 2 * ((tiles + slots - 1) / slots);
-  if (const char* e = getenv("G2_ATTN_SPLIT")) target = atol(e) > 0 ? atol(e) : target;   // measurements
   if (target < 2) target = 2;
   int split_of[AT_MAX_CLS / 2];
   int S = 0;
@@ -760,21 +684,6 @@ AttnPlan make_plan(int BH, int QT, int slots, int cap_pairs, int* n_split) {
 }
 }  // namespace
 
-template <bool kSplit>
-auto pick_kernel(int poly) {
-  // poly 0-4: pairs of every 8 on the FMA pipe; + 8: the streamed softmax
-  switch (poly) {
-    case 2: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[2], false>;
-    case 3: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[3], false>;
-    case 4: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[4], false>;
-    case 8: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[0], true>;
-    case 10: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[2], true>;
-    case 11: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[3], true>;
-    case 12: return attn_fwd_tc_kernel<kSplit, POLY_MASKS[4], true>;
-  }
-  return attn_fwd_tc_kernel<kSplit, POLY_MASKS[0], false>;
-}
-
 size_t attention_scratch_bytes(int B, int T, int H) {
   const size_t QT = ((size_t)T + AT_BQ - 1) / AT_BQ;
   return QT * (size_t)B * H * (ATTN_PART_FLOATS * 4 + ATTN_PAIR_FLAGS * 4);
@@ -790,22 +699,15 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  int poly = 0;
-  if (const char* pe = getenv("G2_ATTN_POLY")) poly = atoi(pe);
-  if (poly < 0 || poly > 12) poly = 0;
-  const auto kfalse = pick_kernel<false>(poly);
-  const auto ktrue = pick_kernel<true>(poly);
+  const auto kfalse = attn_fwd_tc_kernel<false>;
+  const auto ktrue = attn_fwd_tc_kernel<true>;
   if (!attr_set[dev]) {
     cudaError_t e = cudaSuccess;
-    for (int pk = 0; pk < 13 && e == cudaSuccess; ++pk) {
-      void (*ks[2])(CUtensorMap, CUtensorMap, int, int, int, int, float, AttnPlan, unsigned*, int*, float*, int, int*,
-                    float*) = {pick_kernel<false>(pk), pick_kernel<true>(pk)};
-      for (auto k : ks) {
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
-        // two CTAs share an SM only with the largest shared-memory carveout
-        if (e == cudaSuccess)
-          e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-      }
+    for (auto k : {kfalse, ktrue}) {
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+      // two CTAs share an SM only with the largest shared-memory carveout
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     }
     int sms = 0;
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -815,15 +717,12 @@ cudaError_t attention_tc_launch(const void* qkv, void* y, int B, int T, int H, i
     if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&own[dev].part), g_attn_part);
     // the register split must fit in what the launch allocates, or the
     // softmax warps' setmaxnreg.inc would never be granted
-    for (int pk = 0; pk < 13 && e == cudaSuccess; ++pk) {
-      cudaFuncAttributes fa[2];
-      e = cudaFuncGetAttributes(&fa[0], pick_kernel<false>(pk));
-      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[1], pick_kernel<true>(pk));
-      if (e != cudaSuccess) return e;
-      for (const cudaFuncAttributes& f : fa)
-        if (f.numRegs * AT_THREADS < 128 * (REG_SOFTMAX + REG_OTHER)) return cudaErrorInvalidConfiguration;
-    }
+    cudaFuncAttributes fa[2];
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[0], kfalse);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[1], ktrue);
     if (e != cudaSuccess) return e;
+    for (const cudaFuncAttributes& f : fa)
+      if (f.numRegs * AT_THREADS < 128 * (REG_SOFTMAX + REG_OTHER)) return cudaErrorInvalidConfiguration;
     own[dev].cap_pairs = OWN_PAIRS;
     attr_set[dev] = true;
   }

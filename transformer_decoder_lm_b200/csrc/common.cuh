@@ -256,16 +256,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-// 32 lanes x 16 columns of 32-bit words to TMEM.
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
 // Instruction descriptor of tcgen05.mma kind::f16 with a K-major A, an
 // MN-major B (B stored with N contiguous), bf16 inputs, fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
@@ -351,33 +341,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^x on the FMA pipe for a pair of floats in packed arithmetic, for
-// x <= 127 (inputs below -126 give about 2^-126): x = n + f with n the
-// nearest integer (by the 1.5 * 2^23 rounding trick) and f in [-0.5, 0.5];
-// 2^f by a degree-4 polynomial fitted here for relative error (max 2.7e-6 on
-// that interval); 2^n added to the exponent field (the low bits of t hold n
-// in two's complement; the shift into the exponent field wraps in unsigned
-// arithmetic, as intended). An alternative to the SFU for part of a softmax's
-// exponentials.
-__device__ __forceinline__ void ex2_poly_x2(uint64_t x, float& y0, float& y1) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t t = f2_add(xc, magic);
-  const uint64_t fr = f2_sub(xc, f2_sub(t, magic));
-  uint64_t p = f2_fma(f2_pack(9.570068679749966e-3f, 9.570068679749966e-3f), fr,
-                      f2_pack(5.5917806923389435e-2f, 5.5917806923389435e-2f));
-  p = f2_fma(p, fr, f2_pack(2.40247443318367e-1f, 2.40247443318367e-1f));
-  p = f2_fma(p, fr, f2_pack(6.931218504905701e-1f, 6.931218504905701e-1f));
-  p = f2_fma(p, fr, f2_pack(9.999992847442627e-1f, 9.999992847442627e-1f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ float rcp_approx(float x) {
