@@ -423,6 +423,18 @@ def run_kernel(args):
         out = torch.empty(M, C, dtype=bf, device="cuda")
         fn = lambda: G.gpt2_op_layernorm(G.GPT2_BF16, x, g, b, M, C, out)
         flops = 0.0
+    elif k == "train":
+        # one training step's forward and backward of the 124M model at B 4,
+        # T 1024 (gpt2_forward_backward: loss and every weight's gradient)
+        model = G.GPT2Model.from_workload(WL, synthetic.make_weights(WL))
+        grads = model.new_grads()
+        tws = model.new_train_workspace()
+        ids_np = synthetic.make_ids(WL)
+        ids = torch.from_numpy(ids_np).cuda()
+        tg = torch.from_numpy(synthetic.next_token_targets(ids_np)).cuda()
+        loss = torch.empty(1, dtype=torch.float32, device="cuda")
+        fn = lambda: model.forward_backward(ids, tg, grads, tws, loss_out=loss)
+        flops = 3.0 * model_flops(WL)   # forward, then about twice its work for the gradients
     elif k == "decode":
         # one incremental decoding step of the 124M model for 4 sequences at
         # position 1023 (context 1024), after a prefill of positions 0..1022
@@ -479,7 +491,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None,
                     help="run one step alone: lmhead, lmhead_ce (no logits), c_attn, attn_proj, c_fc, mlp_proj, "
-                         "attention, embed, embed_ln (with the first ln_1), layernorm, "
+                         "attention, embed, embed_ln (with the first ln_1), layernorm, train (forward + backward), "
                          "decode (one key/value-cache decoding step, B 4, context 1024)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

@@ -507,12 +507,23 @@ cudaError_t layernorm_bwd_launch(const float* x, const void* gamma, const float*
   float* pb = part + (size_t)blocks * C;
   const bf16* gm = static_cast<const bf16*>(gamma);
   bf16* dbf = static_cast<bf16*>(dx_bf16);
-  cudaError_t e;
+  // the largest shared-memory need (C = 2048) once per device, outside any stream capture
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaError_t e = cudaSuccess;
+  if (!attr_done[dev]) {
+    const int most = 2 * LNB_WARPS * 2048 * (int)sizeof(float);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<13>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
 #define G2_LNB(MV)                                                                                                   \
-  e = cudaFuncSetAttribute(layernorm_bwd_kernel<MV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);        \
-  if (e == cudaSuccess)                                                                                              \
-    e = launch_pdl(layernorm_bwd_kernel<MV>, dim3(blocks), dim3(32 * LNB_WARPS), smem, s, x, gm, dh, dx_in, dx_out, \
-                   dbf, pg, pb, M, C);
+  e = launch_pdl(layernorm_bwd_kernel<MV>, dim3(blocks), dim3(32 * LNB_WARPS), smem, s, x, gm, dh, dx_in, dx_out,   \
+                 dbf, pg, pb, M, C);
   if (C <= 512) {
     G2_LNB(4)
   } else if (C <= 1024) {

@@ -160,8 +160,11 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  pdl_wait();   // the operands and the residual stream come from the previous kernel
-  if (threadIdx.x == 0) pdl_trigger();   // the next kernel may start its set-up as SMs free up
+  // The operands and the residual stream come from the previous kernel:
+  // every thread that touches them waits for it (the producer after it has
+  // requested the first stages of a B operand that no kernel writes, the
+  // weights of the forward pass).
+  if (warp != 0) pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -170,16 +173,34 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;   // per stage: a load was issued / its barrier phase parity
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      auto load_b = [&](uint8_t* sa, uint64_t* bar, int n0, int kb) {
+        if (kBmn) {
+#pragma unroll
+          for (int b = 0; b < BN / 64; ++b) tma_load_2d(sa + L::A_BYTES + b * 8192, &tmB, bar, n0 + b * 64, kb * TC_BK);
+        } else {
+          tma_load_2d(sa + L::A_BYTES, &tmB, bar, kb * TC_BK, n0);
+        }
+      };
+      // B of the first tile's first stages ahead of the wait (fresh stages need no empty wait)
+      const int npre = (args.b_const && (int)blockIdx.x < num_tiles) ? min(nk, TC_STAGES) : 0;
+      for (int kb = 0; kb < npre; ++kb) {
+        mbar_arrive_expect_tx(&full[kb], L::STAGE_BYTES);
+        load_b(smem + kb * L::STAGE_BYTES, &full[kb], ((int)blockIdx.x / m_tiles) * BN, kb);
+      }
+      pdl_wait();
+      pdl_trigger();   // the next kernel may start its set-up as SMs free up
+      bool first = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, first = false) {
         const int m0 = (tile % m_tiles) * TC_BM;
         const int n0 = (tile / m_tiles) * BN;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          const bool pre = first && kb < npre;   // stage already holds B and expects its bytes
+          if (!pre && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * L::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          if (!pre) mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
           // K-major: one box of rows x 64 K; MN-major: 64-wide MN boxes of 64 K rows, 8 KB apart
           if (kAmn) {
 #pragma unroll
@@ -187,13 +208,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           } else {
             tma_load_2d(sa, &tmA, &full[stage], kb * TC_BK, m0);
           }
-          if (kBmn) {
-#pragma unroll
-            for (int b = 0; b < BN / 64; ++b)
-              tma_load_2d(sa + L::A_BYTES + b * 8192, &tmB, &full[stage], n0 + b * 64, kb * TC_BK);
-          } else {
-            tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * TC_BK, n0);
-          }
+          if (!pre) load_b(sa, &full[stage], n0, kb);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == TC_STAGES) {

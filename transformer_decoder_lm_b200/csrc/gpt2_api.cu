@@ -115,6 +115,7 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   a.ldo = ldo;
   a.status = m->status;
   a.gelu_tanh = (m->cfg.flags & GPT2_FLAG_GELU_TANH) ? 1 : 0;
+  a.b_const = 1;   // the Linear weights
   cudaError_t e;
   if (m->bf16 && M <= GEMV_MAX_M) {   // a few rows (decoding): one warp per output column
     e = gemv_bf16_launch(epi, A, W, a, s);
@@ -211,6 +212,7 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     a.part = m->part;
     a.tgt_logit = m->tgt;
     a.status = m->status;
+    a.b_const = 1;   // wte
     int n_tiles;
     if (m->ev_lm_begin) G2_CK(cudaEventRecord(m->ev_lm_begin, s));
     if (m->bf16) {
