@@ -9,9 +9,10 @@
 // file holds the rest:
 //
 //   layernorm_bwd   dx = dx_in + r (g dh - mean(g dh) - xh mean(g dh xh)),
-//                   per-block column partials of dh xh and dh (dgamma, dbeta)
-//   col_partials    per-block column sums of a [M, N] matrix (bias gradients)
-//   col_reduce      sum of the partials over blocks, in a fixed order
+//                   per-block column partials of dh xh and dh (dgamma, dbeta),
+//                   of dx (a residual projection's bias gradient) and of a
+//                   second [M, nz] matrix (a bias gradient of a Linear layer)
+//   lnb_reduce      sum of the partials over blocks, in a fixed order
 //   attn_bwd_dvec   Dv[b, h, i] = sum_d dO[i, d] O[i, d]
 //   attn_bwd        per (sequence, head, 64-key tile): P^T, dP^T, dS^T
 //                   recomputed over the query tiles at and after the key tile,
@@ -50,42 +51,44 @@ __device__ __forceinline__ float4 ld_bf16x4(const bf16* p) {
   return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
 }
 
-constexpr int LNB_WARPS = 4, LNB_ROWS_PER_WARP = 8;
+constexpr int LNB_WARPS = 8, LNB_ROWS_PER_WARP = 2;   // 16 rows per block, two blocks per SM
 constexpr int LNB_ROWS_PER_BLOCK = LNB_WARPS * LNB_ROWS_PER_WARP;
-
-// One warp per row, LNB_ROWS_PER_WARP rows per warp in a fixed order; the
-// row (x, dh) stays in registers. Column partials: each warp accumulates its
-// rows into its own shared-memory slice (lanes own distinct columns), then
-// the block adds the slices in warp order and writes one partial row.
 template <int MAXV>
-__global__ void __launch_bounds__(32 * LNB_WARPS) layernorm_bwd_kernel(
-    const float* __restrict__ x, const bf16* __restrict__ gamma, const float* __restrict__ dh,
-    const float* __restrict__ dx_in, float* __restrict__ dx_out, bf16* __restrict__ dx_bf16,
-    float* __restrict__ part_g, float* __restrict__ part_b, int M, int C) {
-  extern __shared__ float lnb_smem[];   // [2][LNB_WARPS][C]
+__global__ void __launch_bounds__(32 * LNB_WARPS, MAXV <= 6 ? 2 : 1) layernorm_bwd_kernel(const LnBwdArgs a) {
+  extern __shared__ float lnb_smem[];   // [3][LNB_WARPS][C]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = a.C, M = a.M;
   float* sg = lnb_smem + (size_t)warp * C;
   float* sbt = lnb_smem + (size_t)(LNB_WARPS + warp) * C;
+  float* ssum = lnb_smem + (size_t)(2 * LNB_WARPS + warp) * C;
+  const size_t pw = (size_t)3 * C + a.nz;
+  float* prow = a.part + (size_t)blockIdx.x * pw;
   pdl_wait();
   pdl_trigger();
-  for (int c = lane; c < C; c += 32) {
-    sg[c] = 0.f;
-    sbt[c] = 0.f;
+  for (int c = lane * 4; c < C; c += 128) {
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(sg + c) = z4;
+    *reinterpret_cast<float4*>(sbt + c) = z4;
+    *reinterpret_cast<float4*>(ssum + c) = z4;
   }
   __syncwarp();
+  const int r_blk = blockIdx.x * LNB_ROWS_PER_BLOCK;
+  const int r_end = min(M, r_blk + LNB_ROWS_PER_BLOCK);
   for (int rr = 0; rr < LNB_ROWS_PER_WARP; ++rr) {
-    const int row = blockIdx.x * LNB_ROWS_PER_BLOCK + warp * LNB_ROWS_PER_WARP + rr;
-    if (row >= M) break;
-    const float* xr = x + (size_t)row * C;
-    const float* gr = dh + (size_t)row * C;
-    float4 xv[MAXV], gv[MAXV], gm[MAXV];
+    const int row = r_blk + warp * LNB_ROWS_PER_WARP + rr;
+    if (row >= M) continue;
+    const float* xr = a.x + (size_t)row * C;
+    const float* gr = a.dh + (size_t)row * C;
+    const float* dir = a.dx_in ? a.dx_in + (size_t)row * C : nullptr;
+    float4 xv[MAXV], gv[MAXV], gm[MAXV], dv[MAXV];
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
       const int c = (lane + 32 * i) * 4;
       if (c < C) {
         xv[i] = *reinterpret_cast<const float4*>(xr + c);
         gv[i] = *reinterpret_cast<const float4*>(gr + c);
-        gm[i] = ld_bf16x4(gamma + c);
+        gm[i] = ld_bf16x4(a.gamma + c);
+        dv[i] = dir ? *reinterpret_cast<const float4*>(dir + c) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     float s = 0.f;
@@ -97,8 +100,8 @@ __global__ void __launch_bounds__(32 * LNB_WARPS) layernorm_bwd_kernel(
 #pragma unroll
     for (int i = 0; i < MAXV; ++i)
       if ((lane + 32 * i) * 4 < C) {
-        const float a = xv[i].x - mean, b = xv[i].y - mean, c2 = xv[i].z - mean, d = xv[i].w - mean;
-        q += (a * a + b * b) + (c2 * c2 + d * d);
+        const float a0 = xv[i].x - mean, b0 = xv[i].y - mean, c0 = xv[i].z - mean, d0 = xv[i].w - mean;
+        q += (a0 * a0 + b0 * b0) + (c0 * c0 + d0 * d0);
       }
     const float rstd = rsqrtf(warp_sum_f(q) / (float)C + 1e-5f);
     // xh = (x - mean) rstd; gx = dh gamma; means of gx and gx xh
@@ -109,39 +112,23 @@ __global__ void __launch_bounds__(32 * LNB_WARPS) layernorm_bwd_kernel(
       if (c < C) {
         xv[i] = make_float4((xv[i].x - mean) * rstd, (xv[i].y - mean) * rstd, (xv[i].z - mean) * rstd,
                             (xv[i].w - mean) * rstd);
-        const float4 gx = make_float4(gv[i].x * gm[i].x, gv[i].y * gm[i].y, gv[i].z * gm[i].z, gv[i].w * gm[i].w);
-        s1 += (gx.x + gx.y) + (gx.z + gx.w);
-        s2 += (gx.x * xv[i].x + gx.y * xv[i].y) + (gx.z * xv[i].z + gx.w * xv[i].w);
-        // column partials of dgamma (dh xh) and dbeta (dh)
-        float* pg = sg + c;
-        float* pb = sbt + c;
-        pg[0] += gv[i].x * xv[i].x;
-        pg[1] += gv[i].y * xv[i].y;
-        pg[2] += gv[i].z * xv[i].z;
-        pg[3] += gv[i].w * xv[i].w;
-        pb[0] += gv[i].x;
-        pb[1] += gv[i].y;
-        pb[2] += gv[i].z;
-        pb[3] += gv[i].w;
+        gm[i] = make_float4(gv[i].x * gm[i].x, gv[i].y * gm[i].y, gv[i].z * gm[i].z, gv[i].w * gm[i].w);
+        s1 += (gm[i].x + gm[i].y) + (gm[i].z + gm[i].w);
+        s2 += (gm[i].x * xv[i].x + gm[i].y * xv[i].y) + (gm[i].z * xv[i].z + gm[i].w * xv[i].w);
       }
     }
     const float m1 = warp_sum_f(s1) / (float)C, m2 = warp_sum_f(s2) / (float)C;
-    float* dor = dx_out + (size_t)row * C;
-    const float* dir = dx_in ? dx_in + (size_t)row * C : nullptr;
-    bf16* dbr = dx_bf16 ? dx_bf16 + (size_t)row * C : nullptr;
+    float* dor = a.dx_out + (size_t)row * C;
+    bf16* dbr = a.dx_bf16 ? a.dx_bf16 + (size_t)row * C : nullptr;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
       const int c = (lane + 32 * i) * 4;
       if (c < C) {
         float4 d;
-        d.x = rstd * (gv[i].x * gm[i].x - m1 - xv[i].x * m2);
-        d.y = rstd * (gv[i].y * gm[i].y - m1 - xv[i].y * m2);
-        d.z = rstd * (gv[i].z * gm[i].z - m1 - xv[i].z * m2);
-        d.w = rstd * (gv[i].w * gm[i].w - m1 - xv[i].w * m2);
-        if (dir) {
-          const float4 o = *reinterpret_cast<const float4*>(dir + c);
-          d = make_float4(d.x + o.x, d.y + o.y, d.z + o.z, d.w + o.w);
-        }
+        d.x = dv[i].x + rstd * (gm[i].x - m1 - xv[i].x * m2);
+        d.y = dv[i].y + rstd * (gm[i].y - m1 - xv[i].y * m2);
+        d.z = dv[i].z + rstd * (gm[i].z - m1 - xv[i].z * m2);
+        d.w = dv[i].w + rstd * (gm[i].w - m1 - xv[i].w * m2);
         *reinterpret_cast<float4*>(dor + c) = d;
         if (dbr) {
           uint2 u;
@@ -149,73 +136,93 @@ __global__ void __launch_bounds__(32 * LNB_WARPS) layernorm_bwd_kernel(
           u.y = pack_bf16x2(d.z, d.w);
           *reinterpret_cast<uint2*>(dbr + c) = u;
         }
+        // this warp's column partials: dh xh, dh, dx_out
+        float4 pg = *reinterpret_cast<float4*>(sg + c);
+        float4 pb = *reinterpret_cast<float4*>(sbt + c);
+        float4 ps = *reinterpret_cast<float4*>(ssum + c);
+        pg = make_float4(pg.x + gv[i].x * xv[i].x, pg.y + gv[i].y * xv[i].y, pg.z + gv[i].z * xv[i].z,
+                         pg.w + gv[i].w * xv[i].w);
+        pb = make_float4(pb.x + gv[i].x, pb.y + gv[i].y, pb.z + gv[i].z, pb.w + gv[i].w);
+        ps = make_float4(ps.x + d.x, ps.y + d.y, ps.z + d.z, ps.w + d.w);
+        *reinterpret_cast<float4*>(sg + c) = pg;
+        *reinterpret_cast<float4*>(sbt + c) = pb;
+        *reinterpret_cast<float4*>(ssum + c) = ps;
       }
     }
+  }
+  // z: thread t sums the 8-column groups t, t + 256, ... over the block's
+  // rows, 8 row loads in flight at a time, rows added in order
+  const int ngz = a.z ? a.nz / 8 : 0;
+  for (int gz = threadIdx.x; gz < ngz; gz += 32 * LNB_WARPS) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int rb = r_blk; rb < r_end; rb += 8) {
+      const bf16* zp = a.z + (size_t)rb * a.nz + 8 * gz;
+      uint4 u[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (rb + k < r_end) u[k] = __ldg(reinterpret_cast<const uint4*>(zp + (size_t)k * a.nz));
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (rb + k < r_end) {
+          const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[2 * j] += __uint_as_float(w4[j] << 16);
+            acc[2 * j + 1] += __uint_as_float(w4[j] & 0xffff0000u);
+          }
+        }
+    }
+    float* pz = prow + 3 * (size_t)C + 8 * gz;
+    *reinterpret_cast<float4*>(pz) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(pz + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    float a = 0.f, b = 0.f;
+  // the block's partial row: warp slices added in warp order
+  for (int j = threadIdx.x * 4; j < 3 * C; j += blockDim.x * 4) {
+    const int part = j / C, c = j - part * C;
+    const float* src = lnb_smem + (size_t)part * LNB_WARPS * C + c;
+    float4 t = *reinterpret_cast<const float4*>(src);
 #pragma unroll
-    for (int w = 0; w < LNB_WARPS; ++w) {
-      a += lnb_smem[(size_t)w * C + c];
-      b += lnb_smem[(size_t)(LNB_WARPS + w) * C + c];
+    for (int w = 1; w < LNB_WARPS; ++w) {
+      const float4 v = *reinterpret_cast<const float4*>(src + (size_t)w * C);
+      t = make_float4(t.x + v.x, t.y + v.y, t.z + v.z, t.w + v.w);
     }
-    part_g[(size_t)blockIdx.x * C + c] = a;
-    part_b[(size_t)blockIdx.x * C + c] = b;
+    *reinterpret_cast<float4*>(prow + j) = t;
   }
 }
 
-constexpr int COL_ROWS = 128;
-
-// Column sums of rows [blockIdx.y * COL_ROWS, +COL_ROWS) of a [M, N] matrix
-// (bf16 or fp32, row pitch ld); thread = 8 consecutive columns, rows in order.
-template <typename T>
-__global__ void __launch_bounds__(256) col_partials_kernel(const T* __restrict__ a, long long ld, int M, int N,
-                                                           float* __restrict__ part) {
-  const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+// Sums of the partial rows over the blocks: column j of [P, pw] partials,
+// rows p = ty, ty + 16, ... in order by each of the 16 thread rows, then the
+// 16 in order; column j goes to dgamma (j < C), dbeta (< 2C), dsum (< 3C) or dz.
+constexpr int LNR_SLICES = 16;
+__global__ void __launch_bounds__(32 * LNR_SLICES) lnb_reduce_kernel(const float* __restrict__ part, int P, int pw,
+                                                                     int C, float* __restrict__ dgamma,
+                                                                     float* __restrict__ dbeta,
+                                                                     float* __restrict__ dsum, float* __restrict__ dz) {
+  __shared__ float red[LNR_SLICES][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int j = blockIdx.x * 32 + tx;
   pdl_wait();
   pdl_trigger();
-  if (c0 < N) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const int r0 = blockIdx.y * COL_ROWS, r1 = min(M, r0 + COL_ROWS);
-    for (int r = r0; r < r1; ++r) {
-      const T* p = a + (size_t)r * ld + c0;
-      if constexpr (sizeof(T) == 2) {
-        const uint4 u = *reinterpret_cast<const uint4*>(p);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[2 * j] += __uint_as_float(w[j] << 16);
-          acc[2 * j + 1] += __uint_as_float(w[j] & 0xffff0000u);
-        }
-      } else {
-        const float4 u = *reinterpret_cast<const float4*>(p);
-        const float4 v = *reinterpret_cast<const float4*>(p + 4);
-        acc[0] += u.x;
-        acc[1] += u.y;
-        acc[2] += u.z;
-        acc[3] += u.w;
-        acc[4] += v.x;
-        acc[5] += v.y;
-        acc[6] += v.z;
-        acc[7] += v.w;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) part[(size_t)blockIdx.y * N + c0 + j] = acc[j];
+  float s = 0.f;
+  if (j < pw) {
+    const float* p = part + j;
+#pragma unroll 8
+    for (int r = ty; r < P; r += LNR_SLICES) s += p[(size_t)r * pw];
   }
-}
-
-// out[c] = sum over p of part[p, c], p in order.
-__global__ void __launch_bounds__(256) col_reduce_kernel(const float* __restrict__ part, int P, int N,
-                                                         float* __restrict__ out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  pdl_wait();
-  pdl_trigger();
-  if (c < N) {
-    float s = 0.f;
-    for (int p = 0; p < P; ++p) s += part[(size_t)p * N + c];
-    out[c] = s;
+  red[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && j < pw) {
+    float t = red[0][tx];
+#pragma unroll
+    for (int k = 1; k < LNR_SLICES; ++k) t += red[k][tx];
+    if (j < C) dgamma[j] = t;
+    else if (j < 2 * C) dbeta[j - C] = t;
+    else if (j < 3 * C) {
+      if (dsum) dsum[j - 2 * C] = t;
+    } else if (dz) {
+      dz[j - 3 * C] = t;
+    }
   }
 }
 
@@ -494,66 +501,50 @@ __global__ void __launch_bounds__(256) embed_bwd_wpe_kernel(const float* __restr
 }  // namespace
 
 int layernorm_bwd_blocks(int M) { return (M + LNB_ROWS_PER_BLOCK - 1) / LNB_ROWS_PER_BLOCK; }
-int col_sum_blocks(int M) { return (M + COL_ROWS - 1) / COL_ROWS; }
 
-cudaError_t layernorm_bwd_launch(const float* x, const void* gamma, const float* dh, const float* dx_in,
-                                 float* dx_out, void* dx_bf16, float* part, float* dgamma, float* dbeta, int M, int C,
+size_t layernorm_bwd_part_floats(int M, int C, int nz) {
+  return (size_t)layernorm_bwd_blocks(M) * ((size_t)3 * C + (size_t)nz);
+}
+
+cudaError_t layernorm_bwd_launch(const LnBwdArgs& a, float* dgamma, float* dbeta, float* dsum, float* dz,
                                  cudaStream_t s) {
-  if (M <= 0) return cudaSuccess;
-  if (C > 2048 || (C & 3)) return cudaErrorInvalidValue;
-  const int blocks = layernorm_bwd_blocks(M);
-  const size_t smem = (size_t)2 * LNB_WARPS * C * sizeof(float);
-  float* pg = part;
-  float* pb = part + (size_t)blocks * C;
-  const bf16* gm = static_cast<const bf16*>(gamma);
-  bf16* dbf = static_cast<bf16*>(dx_bf16);
+  if (a.M <= 0) return cudaSuccess;
+  if (a.C > 2048 || (a.C & 3) || a.nz < 0 || (a.z && (a.nz % 8)) || (!a.z && a.nz)) return cudaErrorInvalidValue;
+  const int blocks = layernorm_bwd_blocks(a.M);
+  const size_t smem = (size_t)3 * LNB_WARPS * a.C * sizeof(float);
   // the largest shared-memory need (C = 2048) once per device, outside any stream capture
   static bool attr_done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   cudaError_t e = cudaSuccess;
   if (!attr_done[dev]) {
-    const int most = 2 * LNB_WARPS * 2048 * (int)sizeof(float);
+    const int most = 3 * LNB_WARPS * 2048 * (int)sizeof(float);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<13>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(layernorm_bwd_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-#define G2_LNB(MV)                                                                                                   \
-  e = launch_pdl(layernorm_bwd_kernel<MV>, dim3(blocks), dim3(32 * LNB_WARPS), smem, s, x, gm, dh, dx_in, dx_out,   \
-                 dbf, pg, pb, M, C);
-  if (C <= 512) {
+#define G2_LNB(MV) e = launch_pdl(layernorm_bwd_kernel<MV>, dim3(blocks), dim3(32 * LNB_WARPS), smem, s, a);
+  if (a.C <= 512) {
     G2_LNB(4)
-  } else if (C <= 1024) {
+  } else if (a.C <= 768) {
+    G2_LNB(6)
+  } else if (a.C <= 1024) {
     G2_LNB(8)
-  } else if (C <= 1664) {
+  } else if (a.C <= 1664) {
     G2_LNB(13)
   } else {
     G2_LNB(16)
   }
 #undef G2_LNB
   if (e != cudaSuccess) return e;
-  e = launch_pdl(col_reduce_kernel, dim3((C + 255) / 256), dim3(256), 0, s, (const float*)pg, blocks, C, dgamma);
-  if (e == cudaSuccess)
-    e = launch_pdl(col_reduce_kernel, dim3((C + 255) / 256), dim3(256), 0, s, (const float*)pb, blocks, C, dbeta);
-  return e;
-}
-
-cudaError_t col_sum_launch(const void* a, bool a_bf16, long long ld, int M, int N, float* part, float* out,
-                           cudaStream_t s) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
-  if (N % 8) return cudaErrorInvalidValue;
-  const int P = col_sum_blocks(M);
-  const dim3 grid((N / 8 + 255) / 256, P);
-  cudaError_t e = a_bf16 ? launch_pdl(col_partials_kernel<bf16>, grid, dim3(256), 0, s, static_cast<const bf16*>(a),
-                                      ld, M, N, part)
-                         : launch_pdl(col_partials_kernel<float>, grid, dim3(256), 0, s, static_cast<const float*>(a),
-                                      ld, M, N, part);
-  if (e == cudaSuccess)
-    e = launch_pdl(col_reduce_kernel, dim3((N + 255) / 256), dim3(256), 0, s, (const float*)part, P, N, out);
-  return e;
+  const int pw = 3 * a.C + a.nz;
+  return launch_pdl(lnb_reduce_kernel, dim3((pw + 31) / 32), dim3(32 * LNR_SLICES), 0, s, (const float*)a.part, blocks,
+                    pw, a.C,
+                    dgamma, dbeta, dsum, dz);
 }
 
 cudaError_t attention_bwd_launch(const void* qkv, const void* y, const void* dy, const float* lse2, float* Dv,

@@ -1,7 +1,9 @@
 // backward.h - launchers of the backward-pass kernels (internal; backward.cu).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 
 namespace g2 {
 
@@ -9,18 +11,26 @@ namespace g2 {
 // gamma bf16 [C], dh fp32 [M, C] (gradient of the LayerNorm output):
 //   dx_out = dx_in + rstd (g dh - mean(g dh) - xh mean(g dh xh))
 // (dx_in may be NULL, dx_out may equal dx_in; dx_bf16, if not NULL, receives a
-// bf16 copy of dx_out), dgamma = sum_rows dh xh, dbeta = sum_rows dh (fp32 [C]).
-// part: layernorm_bwd_blocks(M) * 2 * C floats of scratch.
+// bf16 copy of dx_out), dgamma = sum_rows dh xh, dbeta = sum_rows dh (fp32
+// [C]); in the same pass dsum = sum_rows dx_out [C] and dz = sum_rows z [nz]
+// of a bf16 matrix z [M, nz] (nz % 8 == 0), each when its pointer is not
+// NULL. All sums add in a fixed order. part: layernorm_bwd_part_floats floats.
+struct LnBwdArgs {
+  const float* x;
+  const __nv_bfloat16* gamma;
+  const float* dh;
+  const float* dx_in;
+  float* dx_out;
+  __nv_bfloat16* dx_bf16;
+  const __nv_bfloat16* z;
+  int nz;
+  float* part;
+  int M, C;
+};
 int layernorm_bwd_blocks(int M);
-cudaError_t layernorm_bwd_launch(const float* x, const void* gamma, const float* dh, const float* dx_in,
-                                 float* dx_out, void* dx_bf16, float* part, float* dgamma, float* dbeta, int M, int C,
+size_t layernorm_bwd_part_floats(int M, int C, int nz);
+cudaError_t layernorm_bwd_launch(const LnBwdArgs& a, float* dgamma, float* dbeta, float* dsum, float* dz,
                                  cudaStream_t s);
-
-// out[c] = sum over the M rows of a [M, N] matrix (bf16 or fp32, row pitch ld
-// elements, N % 8 == 0), added in a fixed order. part: col_sum_blocks(M) * N floats.
-int col_sum_blocks(int M);
-cudaError_t col_sum_launch(const void* a, bool a_bf16, long long ld, int M, int N, float* part, float* out,
-                           cudaStream_t s);
 
 // Attention gradient (bf16, d_head 64): qkv [B, T, 3C] and y [B, T, C] of the
 // forward, dy [B, T, C], lse2 [B, H, T] (per query row: log2 of the softmax

@@ -82,9 +82,7 @@ TrainPlan plan_train(const gpt2_config_t& c, int max_B, int max_T) {
   p.dqkv = o;     o += align256(M * 3 * C * 2);
   p.dq = o;       o += align256(M * C * 4);
   p.dv = o;       o += align256(M * H * 4);
-  const size_t part_ln = (size_t)layernorm_bwd_blocks((int)M) * 2 * C * 4;
-  const size_t part_col = (size_t)col_sum_blocks((int)M) * 4 * C * 4;
-  p.part = o;     o += align256(std::max(part_ln, part_col));
+  p.part = o;     o += align256(layernorm_bwd_part_floats((int)M, (int)C, 4 * (int)C) * 4);
   p.total = o;
   return p;
 }
@@ -240,7 +238,26 @@ int run_train(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B, 
   }
   G2_RC(gm.run(EPI_F32, dz, false, Vp, m->wte, true, C, dh, C, true, M, C, Vp, GemmArgs{}, nullptr, V));   // dhf = dz . wte
   G2_RC(gm.run(EPI_F32, dz, true, Vp, hf, true, C, gr->wte, C, true, V, C, M));            // dwte = dz^T . hf
-  G2_CK(layernorm_bwd_launch(x_fin, m->lnf_g, dh, nullptr, dx, dxb, part, gr->lnf_g, gr->lnf_b, M, C, s));
+  // LayerNorm gradients; each also sums its dx over the rows (the bias
+  // gradient of the residual projection above it) and the bias gradient of
+  // the Linear layer whose output gradient is given as z
+  auto ln_bwd = [&](const float* x, const void* g, const float* dx_in, const void* z, int nz, float* dgamma,
+                    float* dbeta, float* dsum, float* dzsum) {
+    LnBwdArgs a{};
+    a.x = x;
+    a.gamma = static_cast<const bf16*>(g);
+    a.dh = dh;
+    a.dx_in = dx_in;
+    a.dx_out = dx;
+    a.dx_bf16 = static_cast<bf16*>(dxb);
+    a.z = static_cast<const bf16*>(z);
+    a.nz = nz;
+    a.part = part;
+    a.M = M;
+    a.C = C;
+    return layernorm_bwd_launch(a, dgamma, dbeta, dsum, dzsum, s);
+  };
+  G2_CK(ln_bwd(x_fin, m->lnf_g, nullptr, nullptr, 0, gr->lnf_g, gr->lnf_b, gr->mlp_proj_b[L - 1], nullptr));
   for (int l = L - 1; l >= 0; --l) {
     const LayerPtrs& w = m->layers[l];
     const float* x_in = reinterpret_cast<const float*>(layer(l, p.x_in));
@@ -255,20 +272,17 @@ int run_train(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B, 
     ag.gelu_tanh = gelu_tanh;
     G2_RC(gm.run(EPI_DGELU, dxb, false, C, w.mlp_proj_w, true, 4 * C, du, 4 * C, false, M, 4 * C, C, ag));
     G2_RC(gm.run(EPI_F32, dxb, true, C, f, true, 4 * C, gr->mlp_proj_w[l], 4 * C, true, C, 4 * C, M));
-    G2_CK(col_sum_launch(dx, false, C, M, C, part, gr->mlp_proj_b[l], s));
     G2_RC(gm.run(EPI_F32, du, false, 4 * C, w.fc_w, true, C, dh, C, true, M, C, 4 * C));
     G2_RC(gm.run(EPI_F32, du, true, 4 * C, h2, true, C, gr->fc_w[l], C, true, 4 * C, C, M));
-    G2_CK(col_sum_launch(du, true, 4 * C, M, 4 * C, part, gr->fc_b[l], s));
-    G2_CK(layernorm_bwd_launch(x_mid, w.ln2_g, dh, dx, dx, dxb, part, gr->ln2_g[l], gr->ln2_b[l], M, C, s));
+    G2_CK(ln_bwd(x_mid, w.ln2_g, dx, du, 4 * C, gr->ln2_g[l], gr->ln2_b[l], gr->attn_proj_b[l], gr->fc_b[l]));
     // attention: x_mid = x_in + c_proj(attn(c_attn(ln_1(x_in))))
     G2_RC(gm.run(EPI_BIAS, dxb, false, C, w.attn_proj_w, true, C, dy, C, false, M, C, C));
     G2_RC(gm.run(EPI_F32, dxb, true, C, y, true, C, gr->attn_proj_w[l], C, true, C, C, M));
-    G2_CK(col_sum_launch(dx, false, C, M, C, part, gr->attn_proj_b[l], s));
     G2_CK(attention_bwd_launch(qkv, y, dy, lse, dvec, dq, dqkv, B, T, H, C, s));
     G2_RC(gm.run(EPI_F32, dqkv, false, 3 * C, w.attn_w, true, C, dh, C, true, M, C, 3 * C));
     G2_RC(gm.run(EPI_F32, dqkv, true, 3 * C, h1, true, C, gr->attn_w[l], C, true, 3 * C, C, M));
-    G2_CK(col_sum_launch(dqkv, true, 3 * C, M, 3 * C, part, gr->attn_b[l], s));
-    G2_CK(layernorm_bwd_launch(x_in, w.ln1_g, dh, dx, dx, dxb, part, gr->ln1_g[l], gr->ln1_b[l], M, C, s));
+    G2_CK(ln_bwd(x_in, w.ln1_g, dx, dqkv, 3 * C, gr->ln1_g[l], gr->ln1_b[l], l > 0 ? gr->mlp_proj_b[l - 1] : nullptr,
+                 gr->attn_b[l]));
   }
   G2_CK(embed_bwd_launch(ids, dx, gr->wte, gr->wpe, B, T, c.n_ctx, C, V, s));
   return GPT2_OK;
@@ -346,18 +360,26 @@ int gpt2_op_linear_dgrad_gelu(const void* dy, const void* W, const void* u, int 
 
 size_t gpt2_op_layernorm_backward_workspace_bytes(int M, int C) {
   if (M < 1 || C < 4) return 0;
-  return (size_t)layernorm_bwd_blocks(M) * 2 * C * 4;
+  return layernorm_bwd_part_floats(M, C, 0) * 4;
 }
 
 int gpt2_op_layernorm_backward(const float* x, const void* gamma, const float* dh, const float* dx_in, int M, int C,
                                float* dx_out, float* dgamma, float* dbeta, void* workspace, size_t ws_bytes,
                                void* stream) {
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(dh) || (dx_in && !aligned16(dx_in)) || !aligned16(dx_out) ||
-      !dgamma || !dbeta || !workspace || M < 1 || C < 8 || (C % 8) || C > 2048)
+      !dgamma || !dbeta || !aligned16(workspace) || M < 1 || C < 8 || (C % 8) || C > 2048)
     return GPT2_ERR_INVALID_ARG;
   if (ws_bytes < gpt2_op_layernorm_backward_workspace_bytes(M, C)) return GPT2_ERR_WORKSPACE;
-  return layernorm_bwd_launch(x, gamma, dh, dx_in, dx_out, nullptr, static_cast<float*>(workspace), dgamma, dbeta, M,
-                              C, static_cast<cudaStream_t>(stream)) == cudaSuccess
+  LnBwdArgs a{};
+  a.x = x;
+  a.gamma = static_cast<const bf16*>(gamma);
+  a.dh = dh;
+  a.dx_in = dx_in;
+  a.dx_out = dx_out;
+  a.part = static_cast<float*>(workspace);
+  a.M = M;
+  a.C = C;
+  return layernorm_bwd_launch(a, dgamma, dbeta, nullptr, nullptr, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? GPT2_OK
              : GPT2_ERR_CUDA;
 }
