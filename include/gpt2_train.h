@@ -103,10 +103,12 @@ int gpt2_op_attention_train(const void* qkv, int B, int T, int H, int C, void* y
  * attention it differentiates): qkv, y bf16 and lse2 from
  * gpt2_op_attention_train, dy bf16 [B*T, C] -> dqkv bf16 [B*T, 3C] (dq | dk |
  * dv in the column layout of qkv). Scratch:
- * gpt2_op_attention_backward_workspace_bytes. */
+ * gpt2_op_attention_backward_workspace_bytes. status (int32 on the device,
+ * may be NULL): GPT2_ERR_DEVICE_TIMEOUT is or-ed in if a wait inside the
+ * kernel runs out (the kernel then returns early; dqkv is not valid). */
 size_t gpt2_op_attention_backward_workspace_bytes(int B, int T, int H, int C);
 int gpt2_op_attention_backward(const void* qkv, const void* y, const void* dy, const float* lse2, int B, int T, int H,
-                               int C, void* dqkv, void* workspace, size_t ws_bytes, void* stream);
+                               int C, void* dqkv, void* workspace, size_t ws_bytes, int* status, void* stream);
 
 /* Tied lm_head + cross-entropy backward on a final hidden state hf bf16 [M, C]
  * and wte bf16 [V, C] (targets int32 [M], negative = not scored): the mean

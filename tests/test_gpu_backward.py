@@ -154,7 +154,7 @@ def test_attention_backward(G, B, T, H):
     ref_lse2 = (O.logsumexp_last(s)) / math.log(2.0)
     ws = torch.empty(G.gpt2_op_attention_backward_workspace_bytes(B, T, H, C), dtype=torch.uint8, device="cuda")
     dqkv = torch.empty(B * T, 3 * C, dtype=torch.bfloat16, device="cuda")
-    G.gpt2_op_attention_backward(d_qkv, y, dev(dy, "bf16"), lse2, B, T, H, C, dqkv, ws)
+    G.gpt2_op_attention_backward(d_qkv, y, dev(dy, "bf16"), lse2, B, T, H, C, dqkv, ws, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert max_abs(lse2.cpu().numpy(), ref_lse2) <= 1e-3

@@ -99,7 +99,7 @@ def _load():
         "gpt2_op_layernorm_backward": (i, [vp, vp, vp, vp, i, i, vp, vp, vp, vp, sz, vp]),
         "gpt2_op_attention_train": (i, [vp, i, i, i, i, vp, vp, vp, vp]),
         "gpt2_op_attention_backward_workspace_bytes": (sz, [i, i, i, i]),
-        "gpt2_op_attention_backward": (i, [vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]),
+        "gpt2_op_attention_backward": (i, [vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp, vp]),
         "gpt2_op_lmhead_ce_backward_workspace_bytes": (sz, [i, i]),
         "gpt2_op_lmhead_ce_backward": (i, [vp, vp, vp, i, i, i, vp, vp, vp, vp, sz, vp, vp]),
     }
@@ -333,9 +333,9 @@ def gpt2_op_attention_backward_workspace_bytes(B, T, H, C) -> int:
     return int(lib.gpt2_op_attention_backward_workspace_bytes(B, T, H, C))
 
 
-def gpt2_op_attention_backward(qkv, y, dy, lse2, B, T, H, C, dqkv, workspace, stream=None):
+def gpt2_op_attention_backward(qkv, y, dy, lse2, B, T, H, C, dqkv, workspace, status=None, stream=None):
     _check(lib.gpt2_op_attention_backward(_ptr(qkv), _ptr(y), _ptr(dy), _ptr(lse2), B, T, H, C, _ptr(dqkv),
-                                          _ptr(workspace), _nbytes(workspace), _stream(stream)),
+                                          _ptr(workspace), _nbytes(workspace), _ptr(status), _stream(stream)),
            "gpt2_op_attention_backward")
 
 

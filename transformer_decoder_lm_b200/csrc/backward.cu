@@ -14,20 +14,13 @@
 //                   second [M, nz] matrix (a bias gradient of a Linear layer)
 //   lnb_reduce      sum of the partials over blocks, in a fixed order
 //   attn_bwd_dvec   Dv[b, h, i] = sum_d dO[i, d] O[i, d]
-//   attn_bwd        per (sequence, head, 64-key tile): P^T, dP^T, dS^T
-//                   recomputed over the query tiles at and after the key tile,
-//                   dV += P^T dO, dK += dS^T Q, dQ += dS K (fp32 atomics)
 //   dq_finish       dq (scaled, bf16) into the q columns of dqkv
+// (the attention gradient itself is attention_bwd_tc.cu)
 //   embed_bwd       dwte[id] += dx (fp32 atomics), dwpe[t] = sum_b dx[b, t]
 //
 // Every column reduction adds in a fixed order, so those gradients repeat
 // bit for bit; the two atomic sums (dQ over key tiles, wte rows over repeated
 // tokens) do not.
-//
-// The attention kernel runs on mma.sync (m16n8k16 bf16, fp32 accumulation),
-// the register-fragment form of the tensor cores, with the S^T accumulator
-// reused as the A operand of dV and dK (no trip through shared memory) and
-// dS^T transposed through shared memory for dQ.
 #include <math.h>
 
 #include "backward.h"
@@ -252,205 +245,6 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const bf16* __restri
   }
 }
 
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// two bf16 from two rows of a row-major shared array (lo = first)
-__device__ __forceinline__ uint32_t pair_rows(const bf16* lo, const bf16* hi) {
-  return (uint32_t)(*reinterpret_cast<const uint16_t*>(lo)) | ((uint32_t)(*reinterpret_cast<const uint16_t*>(hi)) << 16);
-}
-
-constexpr int AB_T = 64, AB_D = 64, AB_LDS = AB_D + 8;
-
-// Grid (T / 64 key tiles, H, B), 4 warps; warp w owns keys k0 + 16 w .. +15.
-// Longest key tiles (most query tiles after them) first.
-__global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ qkv, const bf16* __restrict__ dO,
-                                                       const float* __restrict__ lse2, const float* __restrict__ Dv,
-                                                       bf16* __restrict__ dqkv, float* __restrict__ dq_acc, int T,
-                                                       int H, int C, float scale_log2, float scale) {
-  __shared__ __align__(16) bf16 Ks[AB_T][AB_LDS];
-  __shared__ __align__(16) bf16 Vs[AB_T][AB_LDS];
-  __shared__ __align__(16) bf16 Qs[AB_T][AB_LDS];
-  __shared__ __align__(16) bf16 dOs[AB_T][AB_LDS];
-  __shared__ __align__(16) bf16 dSs[AB_T][AB_LDS];   // dS^T: [key][query]
-  __shared__ float lse_s[AB_T], dv_s[AB_T];
-  const int kt = blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int k0 = kt * AB_T;
-  const int QT = (T + AB_T - 1) / AB_T;
-  const size_t ld = 3 * (size_t)C;
-  const bf16* base = qkv + (size_t)b * T * ld;
-  const bf16* dob = dO + (size_t)b * T * C + h * AB_D;
-  const float* lb = lse2 + ((size_t)b * H + h) * T;
-  const float* db = Dv + ((size_t)b * H + h) * T;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  constexpr int CH = AB_D / 8;
-  pdl_wait();
-  pdl_trigger();
-
-  for (int i = tid; i < AB_T * CH; i += 128) {
-    const int r = i / CH, c = (i % CH) * 8;
-    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-    if (k0 + r < T) {
-      const bf16* src = base + (size_t)(k0 + r) * ld + h * AB_D + c;
-      kv = *reinterpret_cast<const uint4*>(src + C);
-      vv = *reinterpret_cast<const uint4*>(src + 2 * C);
-    }
-    *reinterpret_cast<uint4*>(&Ks[r][c]) = kv;
-    *reinterpret_cast<uint4*>(&Vs[r][c]) = vv;
-  }
-  __syncthreads();
-  const int wr = warp * 16;
-  uint32_t kf[AB_D / 16][4], vf[AB_D / 16][4];
-#pragma unroll
-  for (int ks = 0; ks < AB_D / 16; ++ks) {
-    kf[ks][0] = *reinterpret_cast<const uint32_t*>(&Ks[wr + g][ks * 16 + 2 * t]);
-    kf[ks][1] = *reinterpret_cast<const uint32_t*>(&Ks[wr + g + 8][ks * 16 + 2 * t]);
-    kf[ks][2] = *reinterpret_cast<const uint32_t*>(&Ks[wr + g][ks * 16 + 2 * t + 8]);
-    kf[ks][3] = *reinterpret_cast<const uint32_t*>(&Ks[wr + g + 8][ks * 16 + 2 * t + 8]);
-    vf[ks][0] = *reinterpret_cast<const uint32_t*>(&Vs[wr + g][ks * 16 + 2 * t]);
-    vf[ks][1] = *reinterpret_cast<const uint32_t*>(&Vs[wr + g + 8][ks * 16 + 2 * t]);
-    vf[ks][2] = *reinterpret_cast<const uint32_t*>(&Vs[wr + g][ks * 16 + 2 * t + 8]);
-    vf[ks][3] = *reinterpret_cast<const uint32_t*>(&Vs[wr + g + 8][ks * 16 + 2 * t + 8]);
-  }
-  float dk[AB_D / 8][4], dv[AB_D / 8][4];
-#pragma unroll
-  for (int i = 0; i < AB_D / 8; ++i) dk[i][0] = dk[i][1] = dk[i][2] = dk[i][3] = dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
-  const int key0 = k0 + wr + g, key1 = key0 + 8;
-
-  for (int qt = kt; qt < QT; ++qt) {
-    const int q0 = qt * AB_T;
-    __syncthreads();   // the previous tile's Q, dO, dS are no longer read
-    for (int i = tid; i < AB_T * CH; i += 128) {
-      const int r = i / CH, c = (i % CH) * 8;
-      uint4 qv = make_uint4(0, 0, 0, 0), ov = make_uint4(0, 0, 0, 0);
-      if (q0 + r < T) {
-        qv = *reinterpret_cast<const uint4*>(base + (size_t)(q0 + r) * ld + h * AB_D + c);
-        ov = *reinterpret_cast<const uint4*>(dob + (size_t)(q0 + r) * C + c);
-      }
-      *reinterpret_cast<uint4*>(&Qs[r][c]) = qv;
-      *reinterpret_cast<uint4*>(&dOs[r][c]) = ov;
-    }
-    if (tid < AB_T) {
-      const bool ok = q0 + tid < T;
-      lse_s[tid] = ok ? lb[q0 + tid] : 0.f;
-      dv_s[tid] = ok ? db[q0 + tid] : 0.f;
-    }
-    __syncthreads();
-
-    // S^T = K Q^T and dP^T = V dO^T: 16 keys x 64 queries per warp
-    float st[AB_T / 8][4], dpt[AB_T / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < AB_T / 8; ++nt) {
-      st[nt][0] = st[nt][1] = st[nt][2] = st[nt][3] = 0.f;
-      dpt[nt][0] = dpt[nt][1] = dpt[nt][2] = dpt[nt][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < AB_D / 16; ++ks) {
-        const uint32_t q_b0 = *reinterpret_cast<const uint32_t*>(&Qs[nt * 8 + g][ks * 16 + 2 * t]);
-        const uint32_t q_b1 = *reinterpret_cast<const uint32_t*>(&Qs[nt * 8 + g][ks * 16 + 2 * t + 8]);
-        mma16816(st[nt], kf[ks], q_b0, q_b1);
-        const uint32_t o_b0 = *reinterpret_cast<const uint32_t*>(&dOs[nt * 8 + g][ks * 16 + 2 * t]);
-        const uint32_t o_b1 = *reinterpret_cast<const uint32_t*>(&dOs[nt * 8 + g][ks * 16 + 2 * t + 8]);
-        mma16816(dpt[nt], vf[ks], o_b0, o_b1);
-      }
-    }
-    // P^T = 2^(s scale_log2 - lse2) where key <= query < T, else 0;
-    // dS^T = P^T (dP^T - Dv); both kept in the accumulator registers
-#pragma unroll
-    for (int nt = 0; nt < AB_T / 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int ql = nt * 8 + 2 * t + (e & 1);
-        const int q = q0 + ql;
-        const int key = e < 2 ? key0 : key1;
-        const float p = (key <= q && q < T) ? ex2_approx(fmaf(st[nt][e], scale_log2, -lse_s[ql])) : 0.f;
-        st[nt][e] = p;
-        dpt[nt][e] = p * (dpt[nt][e] - dv_s[ql]);
-      }
-    }
-    // dV += P^T dO and dK += dS^T Q: A from the accumulators, B = dO or Q
-    // rows (k = query) read column-wise
-#pragma unroll
-    for (int kk = 0; kk < AB_T / 16; ++kk) {
-      uint32_t pa[4], sa[4];
-      pa[0] = pack_bf16x2(st[2 * kk][0], st[2 * kk][1]);
-      pa[1] = pack_bf16x2(st[2 * kk][2], st[2 * kk][3]);
-      pa[2] = pack_bf16x2(st[2 * kk + 1][0], st[2 * kk + 1][1]);
-      pa[3] = pack_bf16x2(st[2 * kk + 1][2], st[2 * kk + 1][3]);
-      sa[0] = pack_bf16x2(dpt[2 * kk][0], dpt[2 * kk][1]);
-      sa[1] = pack_bf16x2(dpt[2 * kk][2], dpt[2 * kk][3]);
-      sa[2] = pack_bf16x2(dpt[2 * kk + 1][0], dpt[2 * kk + 1][1]);
-      sa[3] = pack_bf16x2(dpt[2 * kk + 1][2], dpt[2 * kk + 1][3]);
-      const int qr = kk * 16 + 2 * t;
-#pragma unroll
-      for (int dn = 0; dn < AB_D / 8; ++dn) {
-        const int dc = dn * 8 + g;
-        mma16816(dv[dn], pa, pair_rows(&dOs[qr][dc], &dOs[qr + 1][dc]), pair_rows(&dOs[qr + 8][dc], &dOs[qr + 9][dc]));
-        mma16816(dk[dn], sa, pair_rows(&Qs[qr][dc], &Qs[qr + 1][dc]), pair_rows(&Qs[qr + 8][dc], &Qs[qr + 9][dc]));
-      }
-      // dS^T rows of this warp into shared memory for dQ
-      *reinterpret_cast<uint32_t*>(&dSs[wr + g][kk * 16 + 2 * t]) = sa[0];
-      *reinterpret_cast<uint32_t*>(&dSs[wr + g + 8][kk * 16 + 2 * t]) = sa[1];
-      *reinterpret_cast<uint32_t*>(&dSs[wr + g][kk * 16 + 2 * t + 8]) = sa[2];
-      *reinterpret_cast<uint32_t*>(&dSs[wr + g + 8][kk * 16 + 2 * t + 8]) = sa[3];
-    }
-    __syncthreads();
-    // dQ rows wr..wr+15 of this query tile += dS K over the tile's 64 keys
-    float dq[AB_D / 8][4];
-#pragma unroll
-    for (int i = 0; i < AB_D / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < AB_T / 16; ++kk) {
-      const int kr = kk * 16 + 2 * t;   // key rows of dS^T
-      uint32_t a[4];
-      a[0] = pair_rows(&dSs[kr][wr + g], &dSs[kr + 1][wr + g]);
-      a[1] = pair_rows(&dSs[kr][wr + g + 8], &dSs[kr + 1][wr + g + 8]);
-      a[2] = pair_rows(&dSs[kr + 8][wr + g], &dSs[kr + 9][wr + g]);
-      a[3] = pair_rows(&dSs[kr + 8][wr + g + 8], &dSs[kr + 9][wr + g + 8]);
-#pragma unroll
-      for (int dn = 0; dn < AB_D / 8; ++dn) {
-        const int dc = dn * 8 + g;
-        mma16816(dq[dn], a, pair_rows(&Ks[kr][dc], &Ks[kr + 1][dc]), pair_rows(&Ks[kr + 8][dc], &Ks[kr + 9][dc]));
-      }
-    }
-    const int qa = q0 + wr + g, qb = qa + 8;
-#pragma unroll
-    for (int dn = 0; dn < AB_D / 8; ++dn) {
-      const int col = h * AB_D + dn * 8 + 2 * t;
-      if (qa < T) {
-        float* p = dq_acc + ((size_t)b * T + qa) * C + col;
-        atomicAdd(p, dq[dn][0]);
-        atomicAdd(p + 1, dq[dn][1]);
-      }
-      if (qb < T) {
-        float* p = dq_acc + ((size_t)b * T + qb) * C + col;
-        atomicAdd(p, dq[dn][2]);
-        atomicAdd(p + 1, dq[dn][3]);
-      }
-    }
-  }
-  // dK (scaled) and dV of this warp's 16 keys into dqkv
-  bf16* ob = dqkv + (size_t)b * T * ld + h * AB_D;
-#pragma unroll
-  for (int dn = 0; dn < AB_D / 8; ++dn) {
-    const int col = dn * 8 + 2 * t;
-    if (key0 < T) {
-      *reinterpret_cast<uint32_t*>(ob + (size_t)key0 * ld + C + col) = pack_bf16x2(dk[dn][0] * scale, dk[dn][1] * scale);
-      *reinterpret_cast<uint32_t*>(ob + (size_t)key0 * ld + 2 * C + col) = pack_bf16x2(dv[dn][0], dv[dn][1]);
-    }
-    if (key1 < T) {
-      *reinterpret_cast<uint32_t*>(ob + (size_t)key1 * ld + C + col) = pack_bf16x2(dk[dn][2] * scale, dk[dn][3] * scale);
-      *reinterpret_cast<uint32_t*>(ob + (size_t)key1 * ld + 2 * C + col) = pack_bf16x2(dv[dn][2], dv[dn][3]);
-    }
-  }
-}
-
 // dqkv[:, 0:C] = bf16(dq_acc * scale); 8 columns per thread.
 __global__ void __launch_bounds__(256) dq_finish_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv,
                                                         int M, int C, float scale) {
@@ -548,21 +342,18 @@ cudaError_t layernorm_bwd_launch(const LnBwdArgs& a, float* dgamma, float* dbeta
 }
 
 cudaError_t attention_bwd_launch(const void* qkv, const void* y, const void* dy, const float* lse2, float* Dv,
-                                 float* dq_acc, void* dqkv, int B, int T, int H, int C, cudaStream_t s) {
+                                 float* dq_acc, void* dqkv, int B, int T, int H, int C, int* status, cudaStream_t s) {
+  constexpr int D = 64;   // d_head
   if (B <= 0 || T <= 0) return cudaSuccess;
-  if (C / H != AB_D || C % 8) return cudaErrorInvalidValue;
-  const bf16* q = static_cast<const bf16*>(qkv);
+  if (C / H != D || C % H || C % 8) return cudaErrorInvalidValue;
   const bf16* o = static_cast<const bf16*>(y);
   const bf16* d = static_cast<const bf16*>(dy);
   bf16* out = static_cast<bf16*>(dqkv);
   const int M = B * T;
   cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)M * C * sizeof(float), s);
   if (e == cudaSuccess) e = launch_pdl(attn_bwd_dvec_kernel, dim3((M + 7) / 8), dim3(256), 0, s, d, o, Dv, B, T, H, C);
-  const float scale = (float)(1.0 / sqrt((double)AB_D));
-  const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)AB_D));
-  if (e == cudaSuccess)
-    e = launch_pdl(attn_bwd_kernel, dim3((T + AB_T - 1) / AB_T, H, B), dim3(128), 0, s, q, d, lse2, (const float*)Dv,
-                   out, dq_acc, T, H, C, scale_log2, scale);
+  const float scale = (float)(1.0 / sqrt((double)D));
+  if (e == cudaSuccess) e = attention_bwd_tc_launch(qkv, dy, lse2, Dv, dq_acc, dqkv, B, T, H, C, status, s);
   if (e == cudaSuccess)
     e = launch_pdl(dq_finish_kernel, dim3((unsigned)(((long long)M * C / 8 + 255) / 256)), dim3(256), 0, s,
                    (const float*)dq_acc, out, M, C, scale);

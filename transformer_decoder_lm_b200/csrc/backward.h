@@ -36,9 +36,14 @@ cudaError_t layernorm_bwd_launch(const LnBwdArgs& a, float* dgamma, float* dbeta
 // forward, dy [B, T, C], lse2 [B, H, T] (per query row: log2 of the softmax
 // normaliser of the scores scaled by log2(e)/sqrt(d_head), as the forward
 // kernel wrote it) -> dqkv bf16 [B, T, 3C]. Scratch: Dv fp32 [B, H, T],
-// dq_acc fp32 [B, T, C] (zeroed here).
+// dq_acc fp32 [B, T, C] (zeroed here). A wait that runs out records
+// DEV_TIMEOUT in *status (when not NULL).
 cudaError_t attention_bwd_launch(const void* qkv, const void* y, const void* dy, const float* lse2, float* Dv,
-                                 float* dq_acc, void* dqkv, int B, int T, int H, int C, cudaStream_t s);
+                                 float* dq_acc, void* dqkv, int B, int T, int H, int C, int* status, cudaStream_t s);
+// The tcgen05 kernel of it (attention_bwd_tc.cu): dK, dV into dqkv, dQ
+// (unscaled) added into dq_acc, given Dv.
+cudaError_t attention_bwd_tc_launch(const void* qkv, const void* dy, const float* lse2, const float* Dv, float* dq_acc,
+                                    void* dqkv, int B, int T, int H, int C, int* status, cudaStream_t s);
 
 // Embedding gradient: dwte[ids[m]] += dx[m] (dwte already holds the lm_head
 // term), dwpe[t] = sum_b dx[b, t] for t < T and 0 up to n_ctx.

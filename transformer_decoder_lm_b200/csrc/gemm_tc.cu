@@ -649,18 +649,30 @@ bool make_tmap_out_f32(CUtensorMap* tm, const void* base, uint64_t rows, uint64_
   return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                       uint64_t s2, uint32_t box0, uint32_t box1) {
+namespace {
+bool encode_3d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* base, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1) {
   if (!load_encode()) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((s1 * 2) & 15) || ((s2 * 2) & 15) || !d0 || !d1 || !d2) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((s1 * esize) & 15) || ((s2 * esize) & 15) || !d0 || !d1 || !d2)
+    return false;
   cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {s1 * 2, s2 * 2};
+  cuuint64_t strides[2] = {s1 * (uint64_t)esize, s2 * (uint64_t)esize};
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = g_encode(tm, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                       uint64_t s2, uint32_t box0, uint32_t box1) {
+  return encode_3d(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d0, d1, d2, s1, s2, box0, box1);
+}
+
+bool make_tmap_3d_f32(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                      uint64_t s2, uint32_t box0, uint32_t box1) {
+  return encode_3d(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, d0, d1, d2, s1, s2, box0, box1);
 }
 
 int gemm_tc_n_tiles(int N, int bn) { return (bn / 64) * ((N + bn - 1) / bn); }   // TcLayout::GROUPS per tile

@@ -76,6 +76,9 @@ bool make_tmap_out_f32(CUtensorMap* tm, const void* base, uint64_t rows, uint64_
 // written in boxes of box1 rows x box0 (= 64) columns, 128-byte swizzle.
 bool make_tmap_3d_bf16(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                        uint64_t s2, uint32_t box0, uint32_t box1);
+// The same for fp32 (box0 = 32 columns = 128 bytes).
+bool make_tmap_3d_f32(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                      uint64_t s2, uint32_t box0, uint32_t box1);
 // Column groups of lm_head partials for N columns (two per tile of width bn).
 int gemm_tc_n_tiles(int N, int bn);
 // The lm_head runs with tiles of at least this width.

@@ -278,7 +278,7 @@ int run_train(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B, 
     // attention: x_mid = x_in + c_proj(attn(c_attn(ln_1(x_in))))
     G2_RC(gm.run(EPI_BIAS, dxb, false, C, w.attn_proj_w, true, C, dy, C, false, M, C, C));
     G2_RC(gm.run(EPI_F32, dxb, true, C, y, true, C, gr->attn_proj_w[l], C, true, C, C, M));
-    G2_CK(attention_bwd_launch(qkv, y, dy, lse, dvec, dq, dqkv, B, T, H, C, s));
+    G2_CK(attention_bwd_launch(qkv, y, dy, lse, dvec, dq, dqkv, B, T, H, C, m->status, s));
     G2_RC(gm.run(EPI_F32, dqkv, false, 3 * C, w.attn_w, true, C, dh, C, true, M, C, 3 * C));
     G2_RC(gm.run(EPI_F32, dqkv, true, 3 * C, h1, true, C, gr->attn_w[l], C, true, 3 * C, C, M));
     G2_CK(ln_bwd(x_in, w.ln1_g, dx, dqkv, 3 * C, gr->ln1_g[l], gr->ln1_b[l], l > 0 ? gr->mlp_proj_b[l - 1] : nullptr,
@@ -401,7 +401,7 @@ size_t gpt2_op_attention_backward_workspace_bytes(int B, int T, int H, int C) {
 }
 
 int gpt2_op_attention_backward(const void* qkv, const void* y, const void* dy, const float* lse2, int B, int T, int H,
-                               int C, void* dqkv, void* workspace, size_t ws_bytes, void* stream) {
+                               int C, void* dqkv, void* workspace, size_t ws_bytes, int* status, void* stream) {
   if (!aligned16(qkv) || !aligned16(y) || !aligned16(dy) || !lse2 || !aligned16(dqkv) || !workspace || B < 1 ||
       T < 1 || H < 1 || C % H || (C % 64) || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return GPT2_ERR_INVALID_ARG;
@@ -410,7 +410,7 @@ int gpt2_op_attention_backward(const void* qkv, const void* y, const void* dy, c
   uint8_t* w = static_cast<uint8_t*>(workspace);
   float* Dv = reinterpret_cast<float*>(w);
   float* dq = reinterpret_cast<float*>(w + align256((size_t)B * H * T * 4));
-  return attention_bwd_launch(qkv, y, dy, lse2, Dv, dq, dqkv, B, T, H, C, static_cast<cudaStream_t>(stream)) ==
+  return attention_bwd_launch(qkv, y, dy, lse2, Dv, dq, dqkv, B, T, H, C, status, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? GPT2_OK
              : GPT2_ERR_CUDA;
