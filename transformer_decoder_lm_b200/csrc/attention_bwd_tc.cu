@@ -241,9 +241,10 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS = tmem + TM_ST + lane_off, tDP = tmem + TM_DPT + lane_off;
     const uint32_t sP = smem_u32(smem + AB_OFF_P), sDS = smem_u32(smem + AB_OFF_DS);
-    // this warp's copy of the query tile's L and Dv (read as broadcasts)
-    float* lse_w = reinterpret_cast<float*>(smem + AB_OFF_LSE) + warp * 256;
-    float* dv_w = lse_w + 128;
+    // this warp's copy of the query tile's -L and Dv (read as pair broadcasts)
+    float* nl_w = reinterpret_cast<float*>(smem + AB_OFF_LSE) + warp * 256;
+    float* dv_w = nl_w + 128;
+    const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
     const float* lrow = lse2 + (size_t)bh * T;
     const float* drow = Dv + (size_t)bh * T;
     bool ok = true;
@@ -253,8 +254,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int jq = lane + 32 * m, q = q0 + jq;
-        // queries past T: L = +inf gives P = 0 (their Q, dO rows read as zero)
-        lse_w[jq] = q < T ? lrow[q] : INFINITY;
+        // queries past T: -L = -inf gives P = 0 (their Q, dO rows read as zero)
+        nl_w[jq] = q < T ? -lrow[q] : -INFINITY;
         dv_w[jq] = q < T ? drow[q] : 0.f;
       }
       __syncwarp();
@@ -263,38 +264,56 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         break;
       }
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {   // queries 32c .. 32c + 31 of the tile
+      const bool diag = i == 0;   // the only tile with keys after some of its queries
+      // P, dS of queries 32c .. 32c + 31 as bf16 pairs
+      auto chunk = [&](int c, uint32_t (&pk)[16], uint32_t (&dk)[16]) {
         uint32_t sv[32], dpv[32];
         tmem_ld_32x32b_x32(tS + c * 32, sv);
         tmem_ld_32x32b_x32(tDP + c * 32, dpv);
         tmem_ld_wait();
-        uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float pp[2], dd[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int jq = c * 32 + 2 * e + t;
-            const float p = (kg <= q0 + jq) ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + t]), scale_log2, -lse_w[jq]))
-                                            : 0.f;
-            pp[t] = p;
-            dd[t] = p * (__uint_as_float(dpv[2 * e + t]) - dv_w[jq]);
+          // queries jq, jq + 1 in packed fp32 pairs: P = 2^(s c - L), dS = P (dP - Dv)
+          const int jq = c * 32 + 2 * e;
+          const float2 nl = *reinterpret_cast<const float2*>(nl_w + jq);
+          const float2 dv = *reinterpret_cast<const float2*>(dv_w + jq);
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2,
+                                     f2_pack(nl.x, nl.y));
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (diag) {
+            p0 = kg <= q0 + jq ? p0 : 0.f;
+            p1 = kg <= q0 + jq + 1 ? p1 : 0.f;
           }
-          pk[e] = pack_bf16x2(pp[0], pp[1]);
-          dk[e] = pack_bf16x2(dd[0], dd[1]);
+          const uint64_t p2 = f2_pack(p0, p1);
+          const uint64_t d2 = f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])),
+                                                f2_pack(dv.x, dv.y)));
+          float d0, d1;
+          f2_unpack(d2, d0, d1);
+          pk[e] = pack_bf16x2(p0, p1);
+          dk[e] = pack_bf16x2(d0, d1);
         }
-        if (c == 0 && i > 0 && !mbar_wait(pds_free, (uint32_t)(i - 1) & 1u, abort_flag)) {   // tile i - 1 read them
+      };
+#pragma unroll 1
+      for (int cb = 0; cb < 2; ++cb) {   // the two 64-query blocks of the tile
+        uint32_t pk0[16], dk0[16], pk1[16], dk1[16];
+        chunk(2 * cb, pk0, dk0);
+        chunk(2 * cb + 1, pk1, dk1);
+        // the first block's exponentials run before the wait for the previous
+        // tile's gradient products to release P^T, dS^T
+        if (cb == 0 && i > 0 && !mbar_wait(pds_free, (uint32_t)(i - 1) & 1u, abort_flag)) {
           ok = false;
           break;
         }
-        // row r of the 64-query block c / 2: 16-byte units 4 (c % 2) .. + 3
-        const uint32_t blk = (uint32_t)(c >> 1) * 16384u;
+        // row r of 64-query block cb: 16-byte units 0-3 (first chunk), 4-7
+        const uint32_t blk = (uint32_t)cb * 16384u;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const int u = 4 * (c & 1) + v;
-          st_shared_v4(sw128(sP + blk, r, u), pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          st_shared_v4(sw128(sDS + blk, r, u), dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+          st_shared_v4(sw128(sP + blk, r, v), pk0[4 * v], pk0[4 * v + 1], pk0[4 * v + 2], pk0[4 * v + 3]);
+          st_shared_v4(sw128(sDS + blk, r, v), dk0[4 * v], dk0[4 * v + 1], dk0[4 * v + 2], dk0[4 * v + 3]);
+          st_shared_v4(sw128(sP + blk, r, 4 + v), pk1[4 * v], pk1[4 * v + 1], pk1[4 * v + 2], pk1[4 * v + 3]);
+          st_shared_v4(sw128(sDS + blk, r, 4 + v), dk1[4 * v], dk1[4 * v + 1], dk1[4 * v + 2], dk1[4 * v + 3]);
         }
       }
       if (!ok) break;
