@@ -306,6 +306,34 @@ def run_ours(args):
     tokens_all = M * world
     value = tokens_all / (ms_step / 1000.0)
 
+    # The same forward without the logits output: loss only (lm_head with the
+    # fused log-sum-exp, no logits written) and the trunk only (ln_f output
+    # left in the workspace, no lm_head), timed the same way.
+    def timed_variant(fn):
+        for _ in range(3):
+            fn()
+        barrier()
+        v0 = torch.cuda.Event(enable_timing=True)
+        v1 = torch.cuda.Event(enable_timing=True)
+        v0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        v1.record(stream)
+        barrier()
+        vms = v0.elapsed_time(v1)
+        if world > 1:
+            vms = gdist.max_over_ranks(vms, "cuda")
+        return {"ms_per_step": vms / args.steps, "tokens_per_s": M * world / (vms / args.steps / 1000.0)}
+
+    variants = {
+        "loss_only": timed_variant(lambda: G.gpt2_forward_loss(model.handle, ids, tg, WL.batch, WL.seq, None, loss,
+                                                               None, stream)),
+        "trunk_only": timed_variant(lambda: G.gpt2_forward(model.handle, ids, WL.batch, WL.seq, None, stream)),
+    }
+    rc = model.status()
+    if rc != 0:
+        raise RuntimeError(f"device status after the variants: {G.gpt2_error_string(rc)}")
+
     # e2e: host buffers, copies inside the timed region
     h_ids = torch.from_numpy(ids_np).pin_memory()
     h_tg = torch.from_numpy(tg_np).pin_memory()
@@ -357,6 +385,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h_ids.numel() * 4 + h_tg.numel() * 4),
                 "d2h_bytes_per_step": 4},
         "gpu_launches": int(launches),
+        "variants": variants,
         "clocks": clk,
         "loss": float(loss.item()),
     }
@@ -435,6 +464,18 @@ def run_kernel(args):
         loss = torch.empty(1, dtype=torch.float32, device="cuda")
         fn = lambda: model.forward_backward(ids, tg, grads, tws, loss_out=loss)
         flops = 3.0 * model_flops(WL)   # forward, then about twice its work for the gradients
+    elif k == "attn_bwd":
+        # the attention gradient of one layer (gpt2_op_attention_backward: Dv,
+        # the tcgen05 kernel, the dq scaling) after one training forward
+        qkv, dy = rnd(M, 3 * C), rnd(M, C)
+        y = torch.empty(M, C, dtype=bf, device="cuda")
+        lse2 = torch.empty(WL.batch, H, WL.seq, dtype=torch.float32, device="cuda")
+        G.gpt2_op_attention_train(qkv, WL.batch, WL.seq, H, C, y, lse2)
+        ws = torch.empty(G.gpt2_op_attention_backward_workspace_bytes(WL.batch, WL.seq, H, C), dtype=torch.uint8,
+                         device="cuda")
+        dqkv = torch.empty(M, 3 * C, dtype=bf, device="cuda")
+        fn = lambda: G.gpt2_op_attention_backward(qkv, y, dy, lse2, WL.batch, WL.seq, H, C, dqkv, ws)
+        flops = 2.5 * WL.batch * 2.0 * C * WL.seq * (WL.seq + 1)
     elif k == "decode":
         # one incremental decoding step of the 124M model for 4 sequences at
         # position 1023 (context 1024), after a prefill of positions 0..1022
@@ -491,7 +532,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default=None,
                     help="run one step alone: lmhead, lmhead_ce (no logits), c_attn, attn_proj, c_fc, mlp_proj, "
-                         "attention, embed, embed_ln (with the first ln_1), layernorm, train (forward + backward), "
+                         "attention, attn_bwd (attention gradient), embed, embed_ln (with the first ln_1), layernorm, "
+                         "train (forward + backward), "
                          "decode (one key/value-cache decoding step, B 4, context 1024)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

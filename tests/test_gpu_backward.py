@@ -55,7 +55,10 @@ def report(name, **kw):
     print("GRAD " + json.dumps({"case": name, **kw}), flush=True)
 
 
-LIN_SHAPES = [(200, 192, 320), (1000, 768, 2304), (4096, 768, 3072), (77, 64, 128)]
+# (tokens M, out N, in K); the last two are weight gradients with few output
+# tiles and many tokens, which run as two K halves added into a zeroed output
+LIN_SHAPES = [(200, 192, 320), (1000, 768, 2304), (4096, 768, 3072), (77, 64, 128), (1500, 384, 256),
+              (4096, 768, 768)]
 
 
 @pytest.mark.parametrize("shape", LIN_SHAPES)
@@ -84,6 +87,11 @@ def test_linear_dgrad_and_wgrad(G, shape):
     assert max_abs(g32, rdx) <= 1e-3 * max(1.0, np.abs(rdx).max())
     assert np.all(np.abs(g16 - rdx) <= np.abs(rdx) * 2.0 ** -8 + 1e-3)
     assert max_abs(gw, rdw) <= 1e-3 * max(1.0, np.abs(rdw).max())
+    # a second call gives the same bits (also when the K range is split in two)
+    dw2 = torch.empty_like(dw)
+    G.gpt2_op_linear_wgrad(d_dy, d_x, M, N, K, dw2, st)
+    torch.cuda.synchronize()
+    assert torch.equal(dw, dw2)
 
 
 @pytest.mark.parametrize("tanh_form", [0, 1])

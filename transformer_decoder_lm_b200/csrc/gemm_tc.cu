@@ -130,8 +130,14 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   const int M = args.M, N = args.N;
   const int m_tiles = (M + TC_BM - 1) / TC_BM;
   const int n_tiles = (N + BN - 1) / BN;
-  const int num_tiles = m_tiles * n_tiles;
-  const int nk = (args.K + TC_BK - 1) / TC_BK;   // a K tail past args.K reads as zero (TMA fill)
+  // EPI_F32 with k_split = 2: each output tile is two work items, the K range
+  // halved, both reduce-added into a zeroed output (0 + a + b: the same bits
+  // in either order)
+  const int ks = (EPI == EPI_F32 && args.k_split == 2) ? 2 : 1;
+  const int mn_tiles = m_tiles * n_tiles;
+  const int num_tiles = mn_tiles * ks;
+  const int nk_all = (args.K + TC_BK - 1) / TC_BK;   // a K tail past args.K reads as zero (TMA fill)
+  const int nk = (nk_all + ks - 1) / ks;             // k-blocks per work item (the last may have fewer)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_STAGES; ++s) {
@@ -182,7 +188,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
         }
       };
       // B of the first tile's first stages ahead of the wait (fresh stages need no empty wait)
-      const int npre = (args.b_const && (int)blockIdx.x < num_tiles) ? min(nk, TC_STAGES) : 0;
+      const int npre = (args.b_const && ks == 1 && (int)blockIdx.x < num_tiles) ? min(nk, TC_STAGES) : 0;
       for (int kb = 0; kb < npre; ++kb) {
         mbar_arrive_expect_tx(&full[kb], L::STAGE_BYTES);
         load_b(smem + kb * L::STAGE_BYTES, &full[kb], ((int)blockIdx.x / m_tiles) * BN, kb);
@@ -191,10 +197,12 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
       pdl_trigger();   // the next kernel may start its set-up as SMs free up
       bool first = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, first = false) {
-        const int m0 = (tile % m_tiles) * TC_BM;
-        const int n0 = (tile / m_tiles) * BN;
-        for (int kb = 0; kb < nk; ++kb) {
-          const bool pre = first && kb < npre;   // stage already holds B and expects its bytes
+        const int mn = tile % mn_tiles, kq = tile / mn_tiles;
+        const int m0 = (mn % m_tiles) * TC_BM;
+        const int n0 = (mn / m_tiles) * BN;
+        const int kb0 = kq * nk, kb1 = min(nk_all, kb0 + nk);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const bool pre = first && kb - kb0 < npre;   // stage already holds B and expects its bytes
           if (!pre && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -235,6 +243,8 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
       bool ok = true;
       int it = 0;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int kq = tile / mn_tiles;
+        const int n_kb = min(nk_all, kq * nk + nk) - kq * nk;
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -243,7 +253,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < n_kb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -288,7 +298,8 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      const int mn = tile % mn_tiles;
+      const int m_blk = mn % m_tiles, n_blk = mn / m_tiles;
       const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
       const int row0 = m0 + q * 32;          // first row of this warp
       const int row = row0 + lane;
@@ -448,7 +459,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (EPI == EPI_RESID)
+            if (EPI == EPI_RESID || ks == 2)
               tma_reduce_add_2d(map, sbuf, col0, row0);
             else
               tma_store_2d(map, sbuf, col0, row0);
@@ -590,7 +601,8 @@ cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUten
     return cudaErrorInvalidValue;
   } else {
     using L = TcLayout<BN, EPI>;
-    const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN);
+    const int ks = (EPI == EPI_F32 && a.k_split == 2) ? 2 : 1;
+    const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN) * ks;
     const int grid = std::min(tiles, num_sms);
     if (grid <= 0) return cudaSuccess;
     return launch_pdl(gemm_tc_kernel<BN, EPI, LAYOUT>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, tA, tB, tC,

@@ -59,6 +59,7 @@ struct GemmArgs {
   long long ld_aux;
   const float* row_lse;    // EPI_DLOGITS: natural-log log-sum-exp of each row [M]
   const int* n_scored;     // EPI_DLOGITS: number of rows with a target (device int)
+  int k_split;             // EPI_F32: 2 = the K range in two work items reduce-added into a zeroed output
   int b_const;             // B is written by no kernel of this stream (the forward's weights): its
                            // first stages may be requested before the previous kernel completes
 };

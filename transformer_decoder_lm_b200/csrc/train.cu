@@ -119,6 +119,13 @@ struct Gemm {
     a.out = out;
     a.ldo = ldo;
     a.status = status;
+    // A weight gradient with too few tiles for the SMs and a long K (the
+    // tokens): the K range in two halves, both added into the zeroed output.
+    const long tiles = (long)((M + 127) / 128) * ((N + bn - 1) / bn);
+    if (epi == EPI_F32 && a_mn && b_mn && out_f32 && 2 * tiles <= sms && K >= 1024) {
+      a.k_split = 2;
+      if (cudaMemset2DAsync(out, (size_t)ldo * 4, 0, (size_t)N * 4, M, s) != cudaSuccess) return GPT2_ERR_CUDA;
+    }
     const int layout = (a_mn ? LAYOUT_A_MN : 0) | (b_mn ? LAYOUT_B_MN : 0);
     return gemm_tc_launch(epi, bn, ta, tb, tc, a, sms, s, layout, out_d ? &td : nullptr) == cudaSuccess
                ? GPT2_OK
