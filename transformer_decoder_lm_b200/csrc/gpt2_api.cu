@@ -318,6 +318,44 @@ int run_decode(gpt2_model* m, void* kv_cache, const int32_t* ids, int B, int pos
 
 // =============================================================== public ABI
 
+size_t g2::lmhead_ce_scratch_bytes(int M, int V) {
+  return align256(lmhead_groups_max(V) * (size_t)M * sizeof(float2)) + 2 * align256((size_t)M * 4);
+}
+
+cudaError_t g2::lmhead_ce_launch(bool bf16, const void* hf, const void* wte, const int32_t* targets, int M, int C,
+                                 int V, float* logits, float* token_loss, float* loss_out, void* scratch, int sms,
+                                 int* status, cudaStream_t s) {
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  const size_t part_bytes = align256(lmhead_groups_max(V) * (size_t)M * sizeof(float2));
+  float2* part = reinterpret_cast<float2*>(ws);
+  float* tgt = reinterpret_cast<float*>(ws + part_bytes);
+  float* tok = reinterpret_cast<float*>(ws + part_bytes + align256((size_t)M * 4));
+  GemmArgs a{};
+  a.M = M;
+  a.N = V;
+  a.K = C;
+  a.out = logits;
+  a.ldo = V;
+  a.targets = targets;
+  a.part = part;
+  a.tgt_logit = tgt;
+  a.status = status;
+  int n_groups;
+  cudaError_t e;
+  if (bf16) {
+    const int bn = std::max(gemm_tc_pick_bn(M, V, sms, EPI_LMHEAD), LMHEAD_MIN_BN);
+    n_groups = gemm_tc_n_tiles(V, bn);
+    CUtensorMap ta, tb;
+    if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return cudaErrorInvalidValue;
+    e = gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, ta, a, sms, s);
+  } else {
+    n_groups = (V + SIMT_BN - 1) / SIMT_BN;
+    e = gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(hf), static_cast<const float*>(wte), a, s);
+  }
+  if (e != cudaSuccess) return e;
+  return ce_finish_launch(part, n_groups, tgt, targets, M, V, token_loss ? token_loss : tok, loss_out, status, s);
+}
+
 extern "C" {
 
 size_t gpt2_workspace_bytes(const gpt2_config_t* cfg, int max_B, int max_T) {
@@ -596,7 +634,7 @@ int gpt2_op_attention(int dtype, const void* qkv, int B, int T, int H, int C, vo
 
 size_t gpt2_op_lmhead_ce_workspace_bytes(int dtype, int M, int V) {
   if ((dtype != GPT2_BF16 && dtype != GPT2_FP32) || M < 1 || V < 1) return 0;
-  return align256(lmhead_groups_max(V) * (size_t)M * sizeof(float2)) + 2 * align256((size_t)M * 4);
+  return lmhead_ce_scratch_bytes(M, V);
 }
 
 int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t* targets, int M, int C, int V,
@@ -606,41 +644,14 @@ int gpt2_op_lmhead_ce(int dtype, const void* hf, const void* wte, const int32_t*
       (C % 8) || V < 1 || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return GPT2_ERR_INVALID_ARG;
   if (ws_bytes < gpt2_op_lmhead_ce_workspace_bytes(dtype, M, V)) return GPT2_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t n_tiles_max = lmhead_groups_max(V);
-  float2* part = reinterpret_cast<float2*>(ws);
-  float* tgt = reinterpret_cast<float*>(ws + align256(n_tiles_max * (size_t)M * sizeof(float2)));
-  float* tok = tgt + align256((size_t)M * 4) / 4;
-  GemmArgs a{};
-  a.M = M;
-  a.N = V;
-  a.K = C;
-  a.out = logits_or_null;
-  a.ldo = V;
-  a.targets = targets;
-  a.part = part;
-  a.tgt_logit = tgt;
-  a.status = status;
-  int n_tiles;
+  int sms = 0;
   if (dtype == GPT2_BF16) {
     if (C % 64) return GPT2_ERR_UNSUPPORTED;
-    int sms = 0;
-    int rc = device_setup(nullptr, &sms);
+    const int rc = device_setup(nullptr, &sms);
     if (rc != GPT2_OK) return rc;
-    const int bn = std::max(gemm_tc_pick_bn(M, V, sms, EPI_LMHEAD), LMHEAD_MIN_BN);
-    n_tiles = gemm_tc_n_tiles(V, bn);
-    CUtensorMap ta, tb;
-    if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;
-    if (gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, ta, a, sms, s) != cudaSuccess) return GPT2_ERR_CUDA;
-  } else {
-    n_tiles = (V + SIMT_BN - 1) / SIMT_BN;
-    if (gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(hf), static_cast<const float*>(wte), a, s) !=
-        cudaSuccess)
-      return GPT2_ERR_CUDA;
   }
-  return ce_finish_launch(part, n_tiles, tgt, targets, M, V, token_loss_or_null ? token_loss_or_null : tok, loss_out,
-                          status, s) == cudaSuccess
+  return lmhead_ce_launch(dtype == GPT2_BF16, hf, wte, targets, M, C, V, logits_or_null, token_loss_or_null, loss_out,
+                          workspace, sms, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? GPT2_OK
              : GPT2_ERR_CUDA;
 }

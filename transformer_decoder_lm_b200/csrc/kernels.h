@@ -88,6 +88,16 @@ constexpr int LMHEAD_MIN_BN = 128;
 // of BN columns cover V padded up to a multiple of BN) or per 64-column SIMT
 // tile; at most ceil(V / 64) + 3 either way.
 inline size_t lmhead_groups_max(int V) { return (size_t)((V + 63) / 64) + 3; }
+// The tied lm_head with the fused cross-entropy on caller-provided scratch of
+// lmhead_ce_scratch_bytes(M, V) bytes, 256-byte aligned (partials
+// [groups][M] float2, target logits [M], per-position losses [M]): the launch
+// sequence of gpt2_op_lmhead_ce and gpt2_op_lmhead_ce_noalloc, arguments
+// already checked. bf16: the tcgen05 path (sms = the device's SM count), else
+// the fp32 SIMT path.
+size_t lmhead_ce_scratch_bytes(int M, int V);
+cudaError_t lmhead_ce_launch(bool bf16, const void* hf, const void* wte, const int32_t* targets, int M, int C, int V,
+                             float* logits, float* token_loss, float* loss_out, void* scratch, int sms, int* status,
+                             cudaStream_t s);
 
 // ---- tcgen05 GEMM (bf16) -------------------------------------------------
 // C = A[M,K] . B[N,K]^T with the epilogue `epi`. N % 8 == 0.

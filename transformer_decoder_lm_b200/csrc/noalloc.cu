@@ -18,7 +18,6 @@
 // (on different streams, or from different host threads) race on it; keep
 // them ordered. Nothing in the array has to start at zero: every partial
 // that the finishing kernel reads is written earlier in the same call.
-#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -40,7 +39,6 @@ struct NoallocDevice {
 std::mutex g_mu;
 NoallocDevice g_devices[kMaxDevices];
 
-inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Per-device set-up, done by the first call on each device with that device
 // current: the scratch array's device address, the SM count and the GEMM
@@ -75,47 +73,13 @@ extern "C" int gpt2_op_lmhead_ce_noalloc(int dtype, const void* hf, const void* 
       (reinterpret_cast<uintptr_t>(hf) & 15) || (reinterpret_cast<uintptr_t>(wte) & 15))
     return GPT2_ERR_INVALID_ARG;
   if (dtype == GPT2_BF16 && (C % 64)) return GPT2_ERR_UNSUPPORTED;
-  // Same scratch layout as gpt2_op_lmhead_ce: partials [groups][M] float2,
-  // target logits [M], per-position losses [M].
-  const size_t groups = lmhead_groups_max(V);
-  const size_t part_bytes = align256(groups * (size_t)M * sizeof(float2));
-  const size_t need = part_bytes + 2 * align256((size_t)M * 4);
-  if (need > (size_t)GPT2_NOALLOC_SCRATCH_BYTES) return GPT2_ERR_SCRATCH_LIMIT;
-
+  // the same scratch layout and launches as gpt2_op_lmhead_ce
+  if (lmhead_ce_scratch_bytes(M, V) > (size_t)GPT2_NOALLOC_SCRATCH_BYTES) return GPT2_ERR_SCRATCH_LIMIT;
   NoallocDevice* d = nullptr;
-  int rc = noalloc_setup(&d);
+  const int rc = noalloc_setup(&d);
   if (rc != GPT2_OK) return rc;
-  uint8_t* ws = static_cast<uint8_t*>(d->scratch);
-  float2* part = reinterpret_cast<float2*>(ws);
-  float* tgt = reinterpret_cast<float*>(ws + part_bytes);
-  float* tok = reinterpret_cast<float*>(ws + part_bytes + align256((size_t)M * 4));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-  GemmArgs a{};
-  a.M = M;
-  a.N = V;
-  a.K = C;
-  a.out = logits_or_null;
-  a.ldo = V;
-  a.targets = targets;
-  a.part = part;
-  a.tgt_logit = tgt;
-  a.status = status;
-  int n_groups;
-  if (dtype == GPT2_BF16) {
-    const int bn = std::max(gemm_tc_pick_bn(M, V, d->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
-    n_groups = gemm_tc_n_tiles(V, bn);
-    CUtensorMap ta, tb;
-    if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;
-    if (gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, ta, a, d->num_sms, s) != cudaSuccess) return GPT2_ERR_CUDA;
-  } else {
-    n_groups = (V + SIMT_BN - 1) / SIMT_BN;
-    if (gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(hf), static_cast<const float*>(wte), a, s) !=
-        cudaSuccess)
-      return GPT2_ERR_CUDA;
-  }
-  return ce_finish_launch(part, n_groups, tgt, targets, M, V, token_loss_or_null ? token_loss_or_null : tok, loss_out,
-                          status, s) == cudaSuccess
+  return lmhead_ce_launch(dtype == GPT2_BF16, hf, wte, targets, M, C, V, logits_or_null, token_loss_or_null, loss_out,
+                          d->scratch, d->num_sms, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? GPT2_OK
              : GPT2_ERR_CUDA;
 }
