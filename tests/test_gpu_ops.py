@@ -92,8 +92,11 @@ LINEAR_SHAPES = [
     (128, 200, 64),       # one m-tile, N tail inside a 64-column group
     (515, 776, 256),      # N tail past 768
     (64, 1600, 1600),     # partial m-tile only
-    (5, 2304, 768),       # a few rows: the one-warp-per-column path
-    (16, 776, 3072),      # its largest row count, N tail, long K
+    (5, 2304, 768),       # a few rows: the few-row path (8 rows held, 4 columns per warp)
+    (16, 776, 3072),      # its largest row count, N tail, long K (one column per warp, K streamed)
+    (4, 3072, 768),       # the decoding step's c_fc shape
+    (1, 768, 3072),       # one row, long K
+    (12, 200, 1024),      # 16 rows held, 2 columns per warp, N tail
 ]
 
 

@@ -350,12 +350,13 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const T* __restrict__ 
   }
 }
 
-// bf16 decode, split over the keys: block (h, b, split) takes up to 256
+// bf16 decode, split over the keys: block (h, b, split) takes up to 128
 // cached positions, one per thread for the scores (each key row read with
 // 16-byte loads), then (D/8 column groups) x (256 / (D/8) key classes) for
 // p v with 16-byte loads; it leaves (max, sum, unnormalised o[D]) in `part`.
-// attn_decode_combine_kernel merges the splits in a fixed order.
-constexpr int DEC_KEYS = 256;
+// attn_decode_combine_kernel merges the splits in a fixed order. Both are
+// launched with programmatic dependent launch.
+constexpr int DEC_KEYS = 128;
 
 template <int D>
 __global__ void __launch_bounds__(DEC_KEYS) attn_decode_part_kernel(const bf16* __restrict__ qkv,
@@ -370,12 +371,19 @@ __global__ void __launch_bounds__(DEC_KEYS) attn_decode_part_kernel(const bf16* 
   const int h = blockIdx.x, b = blockIdx.y, sp = blockIdx.z, H = gridDim.x, S = gridDim.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j0 = sp * DEC_KEYS, n = min(len - j0, DEC_KEYS);   // n >= 1
+  const bf16* base = cache + (size_t)b * n_ctx * 2 * C + h * D;   // key row t at base + t * 2C, value at + C
+  pdl_wait();
+  pdl_trigger();
+  // this thread's key row in flight before the query's round trip
+  uint4 kr[DG];
+  if (tid < n) {
+#pragma unroll
+    for (int u = 0; u < DG; ++u) kr[u] = reinterpret_cast<const uint4*>(base + (size_t)(j0 + tid) * 2 * C)[u];
+  }
   if (tid < D) qs[tid] = __bfloat162float(qkv[(size_t)b * 3 * C + h * D + tid]);
   __syncthreads();
-  const bf16* base = cache + (size_t)b * n_ctx * 2 * C + h * D;   // key row t at base + t * 2C, value at + C
   float sc = -INFINITY;
   if (tid < n) {
-    const uint4* kr = reinterpret_cast<const uint4*>(base + (size_t)(j0 + tid) * 2 * C);
     float acc = 0.f;
 #pragma unroll
     for (int u = 0; u < DG; ++u) {
@@ -433,6 +441,8 @@ template <int D>
 __global__ void __launch_bounds__(D) attn_decode_combine_kernel(const float* __restrict__ part, bf16* __restrict__ y,
                                                                 int C, int S) {
   const int h = blockIdx.x, b = blockIdx.y, H = gridDim.x, d = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const float* pp = part + (size_t)(b * H + h) * S * (D + 2);
   float m = -INFINITY;
   for (int s = 0; s < S; ++s) m = fmaxf(m, pp[s * (D + 2)]);
@@ -449,11 +459,13 @@ template <int D>
 cudaError_t decode_split_launch(const void* qkv, const void* cache, void* y, float* part, int B, int H, int C,
                                 int n_ctx, int len, float scale, cudaStream_t s) {
   const int S = (len + DEC_KEYS - 1) / DEC_KEYS;
-  attn_decode_part_kernel<D><<<dim3(H, B, S), DEC_KEYS, 0, s>>>(static_cast<const bf16*>(qkv),
-                                                                static_cast<const bf16*>(cache), part, C, n_ctx, len,
-                                                                scale);
-  attn_decode_combine_kernel<D><<<dim3(H, B), D, 0, s>>>(part, static_cast<bf16*>(y), C, S);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(attn_decode_part_kernel<D>, dim3(H, B, S), dim3(DEC_KEYS), 0, s,
+                             static_cast<const bf16*>(qkv), static_cast<const bf16*>(cache), part, C, n_ctx, len,
+                             scale);
+  if (e == cudaSuccess)
+    e = launch_pdl(attn_decode_combine_kernel<D>, dim3(H, B), dim3(D), 0, s, (const float*)part, static_cast<bf16*>(y),
+                   C, S);
+  return e;
 }
 
 cudaError_t attention_decode_launch(bool bf16_, const void* qkv, const void* cache, void* y, int B, int H, int C,
