@@ -1,7 +1,9 @@
 // gemv.cu - Linear layers for a few rows (M <= GEMV_MAX_M), bf16.
 //
 // y = A W^T + bias with the Linear epilogues of gemm_tc.cu (bias, GELU in the
-// exact erf or the tanh form, residual add into fp32 x), for the decoding
+// exact erf or the tanh form, residual add into fp32 x), optionally with the
+// new key / value columns also written into the key/value cache (the
+// decoding step's c_attn), for the decoding
 // step and other calls with a handful of rows, where a 128-row tensor-core
 // tile would be almost all padding and would leave most SMs idle. The work is
 // bound by reading W once. Each block copies the M rows of A into shared
@@ -29,7 +31,8 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_bf16_kernel(const bf16* 
                                                                     const bf16* __restrict__ W,
                                                                     const bf16* __restrict__ bias, void* out, int M,
                                                                     int N, int K, long long ldo, int gelu_tanh,
-                                                                    int w_const) {
+                                                                    int w_const, bf16* __restrict__ kv,
+                                                                    long long ld_kv, int kv_col0) {
   extern __shared__ uint4 gemv_a[];   // [M][K / 8]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KU = K / 8;
@@ -109,6 +112,8 @@ __global__ void __launch_bounds__(32 * GEMV_WARPS) gemv_bf16_kernel(const bf16* 
           v = gelu_tanh ? 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)))
                         : 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
         static_cast<bf16*>(out)[(size_t)lane * ldo + n] = __float2bfloat16_rn(v);
+        if (EPI == EPI_BIAS && kv != nullptr && n >= kv_col0)
+          kv[(size_t)lane * ld_kv + (n - kv_col0)] = __float2bfloat16_rn(v);
       }
     }
   }
@@ -128,7 +133,8 @@ cudaError_t gemv_one(const bf16* A, const bf16* W, const GemmArgs& a, cudaStream
   }
   const dim3 grid((a.N + GEMV_WARPS * COLS - 1) / (GEMV_WARPS * COLS)), block(32 * GEMV_WARPS);
   return launch_pdl(gemv_bf16_kernel<EPI, MT, COLS, LPC>, grid, block, smem, s, A, W,
-                    static_cast<const bf16*>(a.bias), a.out, a.M, a.N, a.K, a.ldo, a.gelu_tanh, a.b_const);
+                    static_cast<const bf16*>(a.bias), a.out, a.M, a.N, a.K, a.ldo, a.gelu_tanh, a.b_const,
+                    static_cast<bf16*>(a.kv), a.ld_kv, a.kv_col0);
 }
 
 // rows held: 4, 8 or 16; one column per warp (the GPT-2 Linear layers have

@@ -104,9 +104,11 @@ int device_setup(int* dev_out, int* sms_out) {
 namespace {
 
 // One Linear layer of the schedule.
+// extra: the few-row GEMV's cache-append fields, or NULL.
 int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, const void* W, const CUtensorMap* wmaps,
-               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s) {
-  GemmArgs a{};
+               const CUtensorMap* tmC, const void* bias, int M, int N, int K, void* out, long long ldo, cudaStream_t s,
+               const GemmArgs* extra = nullptr) {
+  GemmArgs a = extra ? *extra : GemmArgs{};
   a.M = M;
   a.N = N;
   a.K = K;
@@ -266,6 +268,8 @@ int run_decode(gpt2_model* m, void* kv_cache, const int32_t* ids, int B, int pos
     rc = (expr);                     \
     if (rc != GPT2_OK) return rc;    \
   } while (0)
+  // bf16 with a few rows: the GEMV path, whose c_attn also appends to the cache
+  const bool gemv = m->bf16 && M <= GEMV_MAX_M;
   // x = wte[id] + wpe[pos]: the embedding of one position per row
   const void* wpe_pos = static_cast<const uint8_t*>(m->wpe) + (size_t)pos * C * es;
   G2_CK(embed_launch(m->bf16, ids, m->wte, wpe_pos, m->x, M, 1, C, V, m->status, s));
@@ -274,12 +278,23 @@ int run_decode(gpt2_model* m, void* kv_cache, const int32_t* ids, int B, int pos
     const WeightMaps* W = m->bf16 ? &m->maps[l] : nullptr;
     uint8_t* cl = static_cast<uint8_t*>(kv_cache) + (size_t)l * kv_layer_bytes(m);
     G2_CK(layernorm_launch(m->bf16, m->x, L.ln1_g, L.ln1_b, m->h, M, C, s));
-    G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C,
-                     m->qkv, 3 * C, s));
-    // the new k and v at position pos of each sequence
-    G2_CK(cudaMemcpy2DAsync(cl + (size_t)pos * 2 * C * es, (size_t)c.n_ctx * 2 * C * es,
-                            static_cast<uint8_t*>(m->qkv) + (size_t)C * es, 3 * C * es, 2 * C * es, B,
-                            cudaMemcpyDeviceToDevice, s));
+    if (gemv) {
+      // the c_attn GEMV's k and v columns also go to position pos of each
+      // sequence in the cache
+      GemmArgs e{};
+      e.kv = cl + (size_t)pos * 2 * C * es;
+      e.ld_kv = (long long)c.n_ctx * 2 * C;
+      e.kv_col0 = C;
+      G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C,
+                       m->qkv, 3 * C, s, &e));
+    } else {
+      G2_RC(run_linear(m, EPI_BIAS, m->h, &tm_h, L.attn_w, W ? W->attn : nullptr, &out_qkv, L.attn_b, M, 3 * C, C,
+                       m->qkv, 3 * C, s));
+      // the new k and v at position pos of each sequence
+      G2_CK(cudaMemcpy2DAsync(cl + (size_t)pos * 2 * C * es, (size_t)c.n_ctx * 2 * C * es,
+                              static_cast<uint8_t*>(m->qkv) + (size_t)C * es, 3 * C * es, 2 * C * es, B,
+                              cudaMemcpyDeviceToDevice, s));
+    }
     // the lm_head partials buffer is free until the end of the step: split-key scratch
     G2_CK(attention_decode_launch(m->bf16, m->qkv, cl, m->y, B, H, C, c.n_ctx, pos + 1,
                                   reinterpret_cast<float*>(m->part), (m->plan.tgt - m->plan.part) / sizeof(float), s));

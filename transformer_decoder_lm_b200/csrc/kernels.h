@@ -62,6 +62,10 @@ struct GemmArgs {
   int k_split;             // EPI_F32: 2 = the K range in two work items reduce-added into a zeroed output
   int b_const;             // B is written by no kernel of this stream (the forward's weights): its
                            // first stages may be requested before the previous kernel completes
+  // few-row GEMV only (decoding):
+  void* kv;                // EPI_BIAS: when not NULL, columns n >= kv_col0 are also written as bf16 to
+  long long ld_kv;         // kv[row * ld_kv + n - kv_col0] (the new key and value into the cache)
+  int kv_col0;
 };
 
 // ---- tensor maps (host) -------------------------------------------------
