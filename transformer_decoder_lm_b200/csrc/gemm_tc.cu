@@ -94,16 +94,53 @@ __device__ __forceinline__ void load_bias32_raw(const bf16* bias, int col0, int 
   }
 }
 
-// Derivative of the GELU at the pre-activation u: exact form
-// d/du [u Phi(u)] = Phi(u) + u phi(u); tanh form
-// d/du [u (1 + tanh(k (u + c u^3))) / 2] = (1 + t) / 2 + u (1 - t^2) k (1 + 3 c u^2) / 2.
-__device__ __forceinline__ float gelu_grad(float u, int tanh_form) {
+// Derivative of the GELU at the pre-activation u, on a pair in packed fp32.
+// Exact form: d/du [u Phi(u)] = Phi(u) + u phi(u), with Phi from the same
+// Abramowitz-Stegun 7.1.28 erf as the forward (r ~= erfc(|u|/sqrt2): Phi is
+// 1 - r/2 for u >= 0, r/2 below) and phi(u) = 2^(-u^2 log2(e) / 2) / sqrt(2 pi)
+// on the SFU. Tanh form: d/du [u (1 + t) / 2], t = tanh(v), v = k (u + c u^3):
+// (1 + t) / 2 + u (1 - t^2) k (1 + 3 c u^2) / 2, with (1 + t) / 2 = 1 / (1 +
+// e^(-2v)) from the SFU exponential and reciprocal.
+__device__ __forceinline__ uint64_t gelu_grad_x2(uint64_t u, int tanh_form) {
+  float u0, u1;
+  f2_unpack(u, u0, u1);
   if (tanh_form) {
     const float k = 0.7978845608028654f, c = 0.044715f;
-    const float t = tanhf(k * fmaf(c * u * u, u, u));
-    return 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * k * fmaf(3.f * c, u * u, 1.f);
+    const uint64_t sq = f2_mul(u, u);
+    const uint64_t v = f2_mul(f2_fma(f2_mul(sq, f2_pack(c, c)), u, u), f2_pack(k, k));
+    float v0, v1;
+    f2_unpack(v, v0, v1);
+    // s = (1 + t) / 2 = 1 / (1 + 2^(-2 v log2 e)); 1 - t^2 = 4 s (1 - s)
+    const float s0 = rcp_approx(1.f + ex2_approx(-2.8853900817779268f * v0));
+    const float s1 = rcp_approx(1.f + ex2_approx(-2.8853900817779268f * v1));
+    const uint64_t s2 = f2_pack(s0, s1);
+    const uint64_t one_m_t2 = f2_mul(f2_mul(s2, f2_sub(f2_pack(1.f, 1.f), s2)), f2_pack(4.f, 4.f));
+    // u k (1 + 3 c u^2) / 2
+    const uint64_t w = f2_mul(f2_mul(u, f2_pack(0.5f * k, 0.5f * k)), f2_fma(sq, f2_pack(3.f * c, 3.f * c), f2_pack(1.f, 1.f)));
+    return f2_fma(w, one_m_t2, s2);
   }
-  return 0.5f * (1.f + erff(u * 0.70710678118654752f)) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+  const uint64_t z = f2_mul(f2_pack(fabsf(u0), fabsf(u1)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
+  uint64_t p = f2_fma(z, f2_pack(4.30638e-5f, 4.30638e-5f), f2_pack(2.765672e-4f, 2.765672e-4f));
+  p = f2_fma(z, p, f2_pack(1.520143e-4f, 1.520143e-4f));
+  p = f2_fma(z, p, f2_pack(9.2705272e-3f, 9.2705272e-3f));
+  p = f2_fma(z, p, f2_pack(4.22820123e-2f, 4.22820123e-2f));
+  p = f2_fma(z, p, f2_pack(7.05230784e-2f, 7.05230784e-2f));
+  p = f2_fma(z, p, f2_pack(1.0f, 1.0f));
+  p = f2_mul(p, p);
+  p = f2_mul(p, p);
+  p = f2_mul(p, p);
+  p = f2_mul(p, p);   // ^16
+  float p0, p1;
+  f2_unpack(p, p0, p1);
+  const float hr0 = 0.5f * rcp_approx(p0), hr1 = 0.5f * rcp_approx(p1);   // erfc(|u|/sqrt2) / 2
+  const float Phi0 = u0 >= 0.f ? 1.f - hr0 : hr0, Phi1 = u1 >= 0.f ? 1.f - hr1 : hr1;
+  // u phi(u) = u 2^(-u^2 log2(e) / 2) / sqrt(2 pi)
+  const uint64_t e2 = f2_mul(f2_mul(u, u), f2_pack(-0.72134752044448170f, -0.72134752044448170f));
+  float e0, e1;
+  f2_unpack(e2, e0, e1);
+  const uint64_t uphi = f2_mul(f2_mul(u, f2_pack(0.3989422804014327f, 0.3989422804014327f)),
+                               f2_pack(ex2_approx(e0), ex2_approx(e1)));
+  return f2_add(uphi, f2_pack(Phi0, Phi1));
 }
 
 template <int BN, int EPI, int LAYOUT>
@@ -495,9 +532,12 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float u0 = __uint_as_float(ur[j] << 16), u1 = __uint_as_float(ur[j] & 0xffff0000u);
-              pk[j] = pack_bf16x2(__uint_as_float(v[c][2 * j]) * gelu_grad(u0, args.gelu_tanh),
-                                  __uint_as_float(v[c][2 * j + 1]) * gelu_grad(u1, args.gelu_tanh));
+              const uint64_t u2 = f2_pack(__uint_as_float(ur[j] << 16), __uint_as_float(ur[j] & 0xffff0000u));
+              const uint64_t d2 = f2_mul(f2_pack(__uint_as_float(v[c][2 * j]), __uint_as_float(v[c][2 * j + 1])),
+                                         gelu_grad_x2(u2, args.gelu_tanh));
+              float d0, d1;
+              f2_unpack(d2, d0, d1);
+              pk[j] = pack_bf16x2(d0, d1);
             }
           } else if (EPI == EPI_DLOGITS) {
             // dz = (softmax(z) - onehot(target)) / n_scored on scored rows and
