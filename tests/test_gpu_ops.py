@@ -100,14 +100,25 @@ LINEAR_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("bn", ["64", "128", "192", "256", ""])
-@pytest.mark.parametrize("epi", [0, 1, 2, 3])
-@pytest.mark.parametrize("shape", LINEAR_SHAPES)
-def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
+def pin_gemm(monkeypatch, bn, pair):
+    """Pin the tcgen05 GEMM's tile width ("" = cost model) and whether CTA
+    pairs (256-row tiles over two SMs, opt-in) run ("1") or not ("0")."""
     if bn:
         monkeypatch.setenv("G2_GEMM_BN", bn)
     else:
         monkeypatch.delenv("G2_GEMM_BN", raising=False)
+    monkeypatch.setenv("G2_GEMM_PAIR", pair)
+
+
+# (pair, tile width): a pair's tiles are at least 128 columns wide
+GEMM_PINS = [(p, bn) for p in ("0", "1") for bn in ("64", "128", "192", "256", "") if not (p == "1" and bn == "64")]
+
+
+@pytest.mark.parametrize("pair,bn", GEMM_PINS)
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
+@pytest.mark.parametrize("shape", LINEAR_SHAPES)
+def test_linear_bf16_tcgen05(G, shape, epi, pair, bn, monkeypatch):
+    pin_gemm(monkeypatch, bn, pair)
     M, N, K = shape
     rng = np.random.default_rng(M * 7 + N + K + epi)
     A = bf16_exact(rng, (M, K))
@@ -125,6 +136,37 @@ def test_linear_bf16_tcgen05(G, shape, epi, bn, monkeypatch):
             ref = O.gelu(ref)
         if epi == 3:
             ref = O.gelu_tanh(ref)
+    G.gpt2_op_linear(G.GPT2_BF16, epi, dev(A, "bf16"), dev(W, "bf16"), dev(bias, "bf16"), M, N, K, out, st)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    assert int(st.item()) == 0
+    if epi == 2:
+        assert max_abs(got, ref) <= 1e-4 * max(1.0, math.sqrt(K) / 16)
+    else:
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-4)
+
+
+@pytest.mark.parametrize("pair", ["0", "1"])
+@pytest.mark.parametrize("M,N,K,epi", [(4096, 2304, 768, 0), (4096, 3072, 768, 1), (4096, 768, 768, 2),
+                                       (4096, 768, 3072, 2)])
+def test_linear_bf16_block_shapes(G, M, N, K, epi, pair, monkeypatch):
+    """The four Linear layers of a 124M block at B 4, T 1024 (several waves of
+    tiles per SM or SM pair), with the tile widths the cost model picks."""
+    pin_gemm(monkeypatch, "", pair)
+    rng = np.random.default_rng(M + N + K + epi)
+    A = bf16_exact(rng, (M, K))
+    W = bf16_exact(rng, (N, K), 1.0 / math.sqrt(K))
+    bias = bf16_exact(rng, (N,), 0.1)
+    ref = O.linear(A.astype(np.float64), W.astype(np.float64), bias.astype(np.float64))
+    if epi == 2:
+        x0 = rng.standard_normal((M, N)).astype(np.float32)
+        out = dev(x0, "fp32")
+        ref = ref + x0
+    else:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        if epi == 1:
+            ref = O.gelu(ref)
+    st = status_word()
     G.gpt2_op_linear(G.GPT2_BF16, epi, dev(A, "bf16"), dev(W, "bf16"), dev(bias, "bf16"), M, N, K, out, st)
     torch.cuda.synchronize()
     got = out.float().cpu().numpy()
@@ -209,13 +251,10 @@ def test_attention(G, dtype, B, T, H, C):
 # ------------------------------------------------------- lm_head + cross-entropy
 
 
-@pytest.mark.parametrize("bn", ["64", "128", "192", "256", ""])
-@pytest.mark.parametrize("M,C,V", [(300, 768, 1000), (128, 128, 50257)])
-def test_lmhead_ce_bf16(G, M, C, V, bn, monkeypatch):
-    if bn:
-        monkeypatch.setenv("G2_GEMM_BN", bn)
-    else:
-        monkeypatch.delenv("G2_GEMM_BN", raising=False)
+@pytest.mark.parametrize("pair,bn", GEMM_PINS)
+@pytest.mark.parametrize("M,C,V", [(300, 768, 1000), (128, 128, 50257), (300, 128, 50257)])
+def test_lmhead_ce_bf16(G, M, C, V, pair, bn, monkeypatch):
+    pin_gemm(monkeypatch, bn, pair)
     rng = np.random.default_rng(M + C + V)
     hf = bf16_exact(rng, (M, C))
     wte = bf16_exact(rng, (V, C), 0.05)

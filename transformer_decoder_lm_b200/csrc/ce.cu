@@ -15,13 +15,16 @@
 namespace g2 {
 
 // One block per 32 rows: lane = row, so every load of a partial is a
-// coalesced 256-byte read of one column group for 32 consecutive rows. The 16
-// warps take the column groups round-robin, each warp with 4 independent
-// running (max, sum) pairs (groups 16 a + warp for a = j mod 4) so that the
-// merge chains overlap; the pairs are merged in a fixed order, per warp and
-// then across warps through shared memory (deterministic). Rescaling uses
+// coalesced 256-byte read of one column group for 32 consecutive rows. The 32
+// warps take the column groups round-robin, each warp with 8 independent
+// running (max, sum) pairs (groups 32 a + warp for a = j mod 8) whose loads
+// are all issued before any merge, so a warp has 8 reads in flight and the
+// ~25 groups of a 50257-column vocabulary take about three memory round
+// trips; the pairs are merged in a fixed order, per warp and then across
+// warps through shared memory (deterministic). Rescaling uses
 // exp(d) = 2^(d log2 e) on the SFU.
-constexpr int CE_WARPS = 16;
+constexpr int CE_WARPS = 32;
+constexpr int CE_LOADS = 8;
 
 __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
   if (m2 == -INFINITY) return;   // a column group with no valid column
@@ -40,24 +43,28 @@ __global__ void __launch_bounds__(32 * CE_WARPS) ce_rows_kernel(const float2* __
   const int row = blockIdx.x * 32 + lane;
   pdl_wait();
   pdl_trigger();
-  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, s[4] = {0.f, 0.f, 0.f, 0.f};
+  float m[CE_LOADS], s[CE_LOADS];
+#pragma unroll
+  for (int a = 0; a < CE_LOADS; ++a) {
+    m[a] = -INFINITY;
+    s[a] = 0.f;
+  }
   if (row < M) {
-    int i = warp;
-    for (; i + 3 * CE_WARPS < n_tiles; i += 4 * CE_WARPS) {
-      float2 p[4];
+    for (int i = warp; i < n_tiles; i += CE_LOADS * CE_WARPS) {
+      float2 p[CE_LOADS];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) p[a] = part[(size_t)(i + a * CE_WARPS) * M + row];
+      for (int a = 0; a < CE_LOADS; ++a) {
+        const int g = i + a * CE_WARPS;
+        p[a] = g < n_tiles ? part[(size_t)g * M + row] : make_float2(-INFINITY, 0.f);
+      }
 #pragma unroll
-      for (int a = 0; a < 4; ++a) lse_merge(m[a], s[a], p[a].x, p[a].y);
-    }
-    for (int a = 0; i < n_tiles; i += CE_WARPS, ++a) {
-      const float2 p = part[(size_t)i * M + row];
-      lse_merge(m[a], s[a], p.x, p.y);
+      for (int a = 0; a < CE_LOADS; ++a) lse_merge(m[a], s[a], p[a].x, p[a].y);
     }
   }
-  lse_merge(m[0], s[0], m[1], s[1]);
-  lse_merge(m[2], s[2], m[3], s[3]);
-  lse_merge(m[0], s[0], m[2], s[2]);
+#pragma unroll
+  for (int w = 1; w < CE_LOADS; w *= 2)
+#pragma unroll
+    for (int a = 0; a < CE_LOADS; a += 2 * w) lse_merge(m[a], s[a], m[a + w], s[a + w]);
   sm_m[warp][lane] = m[0];
   sm_s[warp][lane] = s[0];
   __syncthreads();

@@ -52,7 +52,8 @@ namespace g2 {
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
 constexpr int TC_STAGES = 4;
-template <int BN, int EPI>
+constexpr int TC_SMEM_MAX = 232448;   // dynamic shared memory per block (227 KB)
+template <int BN, int EPI, int CG = 1>
 struct TcLayout {
   // Each epilogue warp owns 32 rows (one TMEM lane quadrant) x COLS_PER_WARP
   // columns: 64 (BN / 16 warps), or half the tile (8 warps; BN = 128, 256) for the lm_head
@@ -65,17 +66,24 @@ struct TcLayout {
   // or 8 logits rows x 64 fp32 (2 KB)
   static constexpr bool F32_OUT = EPI == EPI_RESID || EPI == EPI_F32;
   static constexpr int STAGE_BUF_BYTES = F32_OUT ? 4096 : 2048;
+  static constexpr int EPI_BYTES = EPI_WARPS * STAGE_BUF_BYTES;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
-  static constexpr int B_BYTES = BN * TC_BK * 2;
+  // CTA pair (CG = 2): each CTA stages half of the tile's BN rows of B
+  static constexpr int B_ROWS = BN / CG;
+  static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int EPI_OFFSET = TC_STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_WARPS * STAGE_BUF_BYTES;
-  static constexpr int NUM_BARS = 2 * TC_STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
+  // a single CTA keeps a 4-deep ring; a pair's smaller stages buy up to 6
+  static constexpr int STAGES_FIT = (TC_SMEM_MAX - 1024 - 256 - EPI_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = CG == 1 ? TC_STAGES : (STAGES_FIT < 6 ? STAGES_FIT : 6);
+  static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
   static constexpr int SMEM_BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;   // + holders, 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
   static constexpr int CHUNKS = COLS_PER_WARP / 32;
   static constexpr int GROUPS = BN / 64;   // lm_head: 64-column log-sum-exp groups per tile
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(SMEM_BYTES <= TC_SMEM_MAX, "shared memory budget");
+  static_assert(STAGES >= 2 && STAGE_BYTES % 1024 == 0, "ring of 1 KB-aligned stages");
   static_assert(BN % COLS_PER_WARP == 0 && COLS_PER_WARP % 64 == 0, "whole 64-column groups per warp");
 };
 
@@ -143,20 +151,27 @@ __device__ __forceinline__ uint64_t gelu_grad_x2(uint64_t u, int tanh_form) {
   return f2_add(uphi, f2_pack(Phi0, Phi1));
 }
 
-template <int BN, int EPI, int LAYOUT>
-__global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
+// CG = 2: a CTA pair (cluster of two) computes 256 x BN tiles with one
+// tcgen05.mma of M = 256 issued by the leader (cluster rank 0). Each CTA
+// stages its 128 rows of A and half (BN / 2 rows) of B, so per SM the TMA
+// writes and the tensor core's shared-memory reads per FLOP drop by a
+// third at BN = 256; each CTA's epilogue drains its own 128 accumulator rows.
+template <int BN, int EPI, int LAYOUT, int CG>
+__global__ void __launch_bounds__(TcLayout<BN, EPI, CG>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const GemmArgs args) {
-  using L = TcLayout<BN, EPI>;
+  using L = TcLayout<BN, EPI, CG>;
   constexpr bool kLM = EPI == EPI_LMHEAD || EPI == EPI_LMHEAD_LOGITS;
   constexpr bool kAmn = (LAYOUT & LAYOUT_A_MN) != 0, kBmn = (LAYOUT & LAYOUT_B_MN) != 0;
   constexpr bool kGelu = EPI == EPI_GELU || EPI == EPI_GELU_SAVE;
+  constexpr bool kPair = CG == 2;
+  static_assert(!kPair || (!kAmn && !kBmn), "CTA pairs read K-major operands");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFFSET);
-  uint64_t* empty = full + TC_STAGES;
-  uint64_t* tfull = empty + TC_STAGES;
+  uint64_t* empty = full + L::STAGES;
+  uint64_t* tfull = empty + L::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -165,7 +180,13 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int M = args.M, N = args.N;
-  const int m_tiles = (M + TC_BM - 1) / TC_BM;
+  // rank in the pair (the leader issues the MMAs) and the work walker: one
+  // per CTA, or one per pair
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int walker = kPair ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int n_walkers = kPair ? (int)cluster_count_x() : (int)gridDim.x;
+  const int m_tiles = (M + TC_BM * CG - 1) / (TC_BM * CG);
   const int n_tiles = (N + BN - 1) / BN;
   // EPI_F32 with k_split = 2: each output tile is two work items, the K range
   // halved, both reduce-added into a zeroed output (0 + a + b: the same bits
@@ -177,13 +198,13 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   const int nk = (nk_all + ks - 1) / ks;             // k-blocks per work item (the last may have fewer)
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) {
+    for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], L::EPI_WARPS);
+      mbar_init(&tempty[b], L::EPI_WARPS * CG);   // a pair: both CTAs' epilogue warps free the leader's MMA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -196,11 +217,17 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     if (EPI == EPI_GELU_SAVE) tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, L::TMEM_COLS);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(tmem_holder, L::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, L::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();   // the peer's barriers are initialised before any load or arrive targets them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   // The operands and the residual stream come from the previous kernel:
@@ -216,27 +243,38 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;   // per stage: a load was issued / its barrier phase parity
       bool ok = true;
-      auto load_b = [&](uint8_t* sa, uint64_t* bar, int n0, int kb) {
+      // a pair counts both CTAs' bytes on the leader's full barrier
+      const uint32_t full_leader = kPair ? mapa_shared(smem_u32(full), 0) : 0u;
+      auto load_2d = [&](void* dst, const CUtensorMap* tm, int s, int c0, int c1) {
+        if (kPair)
+          tma_load_2d_pair(dst, tm, full_leader + 8u * s, c0, c1);
+        else
+          tma_load_2d(dst, tm, &full[s], c0, c1);
+      };
+      auto expect = [&](int s) {
+        if (leader) mbar_arrive_expect_tx(&full[s], CG * L::STAGE_BYTES);
+      };
+      auto load_b = [&](uint8_t* sa, int s, int n0, int kb) {
         if (kBmn) {
 #pragma unroll
-          for (int b = 0; b < BN / 64; ++b) tma_load_2d(sa + L::A_BYTES + b * 8192, &tmB, bar, n0 + b * 64, kb * TC_BK);
+          for (int b = 0; b < BN / 64; ++b) load_2d(sa + L::A_BYTES + b * 8192, &tmB, s, n0 + b * 64, kb * TC_BK);
         } else {
-          tma_load_2d(sa + L::A_BYTES, &tmB, bar, kb * TC_BK, n0);
+          load_2d(sa + L::A_BYTES, &tmB, s, kb * TC_BK, n0);
         }
       };
       // B of the first tile's first stages ahead of the wait (fresh stages need no empty wait)
-      const int npre = (args.b_const && ks == 1 && (int)blockIdx.x < num_tiles) ? min(nk, TC_STAGES) : 0;
+      const int npre = (args.b_const && ks == 1 && walker < num_tiles) ? min(nk, L::STAGES) : 0;
       for (int kb = 0; kb < npre; ++kb) {
-        mbar_arrive_expect_tx(&full[kb], L::STAGE_BYTES);
-        load_b(smem + kb * L::STAGE_BYTES, &full[kb], ((int)blockIdx.x / m_tiles) * BN, kb);
+        expect(kb);
+        load_b(smem + kb * L::STAGE_BYTES, kb, (walker / m_tiles) * BN + (int)rank * L::B_ROWS, kb);
       }
       pdl_wait();
       pdl_trigger();   // the next kernel may start its set-up as SMs free up
       bool first = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, first = false) {
+      for (int tile = walker; tile < num_tiles && ok; tile += n_walkers, first = false) {
         const int mn = tile % mn_tiles, kq = tile / mn_tiles;
-        const int m0 = (mn % m_tiles) * TC_BM;
-        const int n0 = (mn / m_tiles) * BN;
+        const int m0 = ((mn % m_tiles) * CG + (int)rank) * TC_BM;
+        const int n0 = (mn / m_tiles) * BN + (int)rank * L::B_ROWS;
         const int kb0 = kq * nk, kb1 = min(nk_all, kb0 + nk);
         for (int kb = kb0; kb < kb1; ++kb) {
           const bool pre = first && kb - kb0 < npre;   // stage already holds B and expects its bytes
@@ -245,18 +283,18 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
             break;
           }
           uint8_t* sa = smem + stage * L::STAGE_BYTES;
-          if (!pre) mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          if (!pre) expect(stage);
           // K-major: one box of rows x 64 K; MN-major: 64-wide MN boxes of 64 K rows, 8 KB apart
           if (kAmn) {
 #pragma unroll
-            for (int b = 0; b < TC_BM / 64; ++b) tma_load_2d(sa + b * 8192, &tmA, &full[stage], m0 + b * 64, kb * TC_BK);
+            for (int b = 0; b < TC_BM / 64; ++b) load_2d(sa + b * 8192, &tmA, stage, m0 + b * 64, kb * TC_BK);
           } else {
-            tma_load_2d(sa, &tmA, &full[stage], kb * TC_BK, m0);
+            load_2d(sa, &tmA, stage, kb * TC_BK, m0);
           }
-          if (!pre) load_b(sa, &full[stage], n0, kb);
+          if (!pre) load_b(sa, stage, n0, kb);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == TC_STAGES) {
+          if (++stage == L::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -266,20 +304,24 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
         record_error(args.status, DEV_TIMEOUT);
         *abort_flag = 1;
       }
-      // Let every issued copy land before the CTA can exit (bounded).
+      // Let every issued copy land before the CTA can exit (bounded). A
+      // pair's copies all complete on the leader's barriers: the leader
+      // waits for both CTAs', and the closing cluster barrier keeps the
+      // peer resident until then.
       volatile int no_abort = 0;
-      for (int s = 0; s < TC_STAGES; ++s)
-        if (issued & (1u << s)) mbar_wait(&full[s], (issued_parity >> s) & 1u, &no_abort);
+      if (leader)
+        for (int s = 0; s < L::STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait(&full[s], (issued_parity >> s) & 1u, &no_abort);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32_major(TC_BM, BN, kAmn, kBmn);
+    if (lane == 0 && leader) {
+      constexpr uint32_t IDESC = idesc_bf16_f32_major(TC_BM * CG, BN, kAmn, kBmn);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = walker; tile < num_tiles && ok; tile += n_walkers, ++it) {
         const int kq = tile / mn_tiles;
         const int n_kb = min(nk_all, kq * nk + nk) - kq * nk;
         const int acc = it & 1;
@@ -303,23 +345,35 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
             const uint64_t adesc = kAmn ? sdesc_mn_sw128(sa + k * 2048, 8192) : sdesc_kmajor_sw128(sa) + 2 * k;
             const uint64_t bdesc =
                 kBmn ? sdesc_mn_sw128(sa + L::A_BYTES + k * 2048, 8192) : sdesc_kmajor_sw128(sa + L::A_BYTES) + 2 * k;
-            mma_bf16_ss(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
+            if (kPair)
+              mma_bf16_ss_pair(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
+            else
+              mma_bf16_ss(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
           }
-          mma_commit(&empty[stage]);
-          if (++stage == TC_STAGES) {
+          if (kPair)
+            mma_commit_pair_both(&empty[stage]);   // frees the stage in both CTAs
+          else
+            mma_commit(&empty[stage]);
+          if (++stage == L::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull[acc]);
+        if (kPair)
+          mma_commit_pair_both(&tfull[acc]);
+        else
+          mma_commit(&tfull[acc]);
       }
       if (!ok) {
         record_error(args.status, DEV_TIMEOUT);
         *abort_flag = 1;
       }
       // Every MMA issued above has completed once `drain` flips.
-      mma_commit(drain);
+      if (kPair)
+        mma_commit_pair(drain);
+      else
+        mma_commit(drain);
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
@@ -331,13 +385,21 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
     const uint32_t sb = smem_u32(sbuf);
     constexpr float LOG2E = 1.4426950408889634f;
     bool store_pending = false;
+    // the accumulator buffers are handed back to the (leader's) MMA warp
+    const uint32_t tempty_leader = kPair ? mapa_shared(smem_u32(tempty), 0) : 0u;
+    auto release_acc = [&](int acc) {
+      if (kPair)
+        mbar_arrive_cluster(tempty_leader + 8u * acc);
+      else
+        mbar_arrive(&tempty[acc]);
+    };
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = walker; tile < num_tiles; tile += n_walkers, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       const int mn = tile % mn_tiles;
       const int m_blk = mn % m_tiles, n_blk = mn / m_tiles;
-      const int m0 = m_blk * TC_BM, n0 = n_blk * BN;
+      const int m0 = (m_blk * CG + (int)rank) * TC_BM, n0 = n_blk * BN;
       const int row0 = m0 + q * 32;          // first row of this warp
       const int row = row0 + lane;
       const bool row_ok = row < M;
@@ -365,7 +427,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (lane == 0) release_acc(acc);
       }
 
       if (kLM) {
@@ -461,7 +523,7 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (lane == 0) release_acc(acc);
         const bf16* bias_p = static_cast<const bf16*>(args.bias);
         // EPI_DLOGITS: this row's target, log-sum-exp (log2 units) and 1 / scored rows
         int d_tgt = -1;
@@ -586,9 +648,16 @@ __global__ void __launch_bounds__(TcLayout<BN, EPI>::THREADS, 1)
   }
 
   __syncthreads();
+  // A pair: the leader's MMAs (which read the peer's shared memory and write
+  // its TMEM) have drained, and the peer's arrivals on the leader's
+  // barriers have landed, before either CTA frees TMEM or exits.
+  if (kPair) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::TMEM_COLS);
+    if (kPair)
+      tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
 }
 
@@ -622,11 +691,15 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
 }
 
 
-// The fp32 epilogues' 4 KB staging per warp does not fit next to the ring at
-// BN = 256 (gemm_tc_pick_bn never picks it there). The backward layouts are
-// instantiated only with the epilogues the backward pass uses.
-template <int BN, int EPI, int LAYOUT>
+// The fp32 epilogues' 4 KB staging per warp does not fit next to a single
+// CTA's ring at BN = 256 (gemm_tc_pick never picks it there). The backward
+// layouts are instantiated only with the epilogues the backward pass uses;
+// CTA pairs with K-major operands, 128 to 256 columns and the forward (and
+// logits-gradient) epilogues.
+template <int BN, int EPI, int LAYOUT, int CG>
 constexpr bool tc_supported() {
+  if (CG == 2)
+    return LAYOUT == LAYOUT_KK && BN >= 128 && EPI != EPI_F32 && EPI != EPI_DGELU;
   if ((EPI == EPI_RESID || EPI == EPI_F32) && BN == 256) return false;
   if (LAYOUT == LAYOUT_B_MN) return EPI == EPI_BIAS || EPI == EPI_F32 || EPI == EPI_DGELU;
   if (LAYOUT == LAYOUT_MN_MN) return EPI == EPI_F32;
@@ -634,54 +707,99 @@ constexpr bool tc_supported() {
   return EPI != EPI_DGELU && EPI != EPI_F32;
 }
 
-template <int BN, int EPI, int LAYOUT>
+// Clusters of two that fit on the device at once (queried once per kernel).
+template <typename Kern>
+int pair_slots(Kern kern, int threads, int smem, int num_sms) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms / 2));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = num_sms / 2;
+  }
+  return std::min(n, num_sms / 2);
+}
+
+template <int BN, int EPI, int LAYOUT, int CG>
 cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC, const CUtensorMap& tD,
                        const GemmArgs& a, int num_sms, cudaStream_t s) {
-  if constexpr (!tc_supported<BN, EPI, LAYOUT>()) {
+  if constexpr (!tc_supported<BN, EPI, LAYOUT, CG>()) {
     return cudaErrorInvalidValue;
   } else {
-    using L = TcLayout<BN, EPI>;
+    using L = TcLayout<BN, EPI, CG>;
+    auto kern = gemm_tc_kernel<BN, EPI, LAYOUT, CG>;
     const int ks = (EPI == EPI_F32 && a.k_split == 2) ? 2 : 1;
-    const int tiles = ((a.M + TC_BM - 1) / TC_BM) * ((a.N + BN - 1) / BN) * ks;
-    const int grid = std::min(tiles, num_sms);
-    if (grid <= 0) return cudaSuccess;
-    return launch_pdl(gemm_tc_kernel<BN, EPI, LAYOUT>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, tA, tB, tC,
-                      tD, a);
+    const int tiles = ((a.M + TC_BM * CG - 1) / (TC_BM * CG)) * ((a.N + BN - 1) / BN) * ks;
+    if (CG == 1) {
+      const int grid = std::min(tiles, num_sms);
+      if (grid <= 0) return cudaSuccess;
+      return launch_pdl(kern, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, s, tA, tB, tC, tD, a);
+    }
+    static const int slots = pair_slots(kern, L::THREADS, L::SMEM_BYTES, num_sms);
+    const int pairs = std::min(tiles, slots);
+    if (pairs <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(L::THREADS);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, tA, tB, tC, tD, a);
   }
 }
 
-template <int BN, int EPI, int LAYOUT>
+template <int BN, int EPI, int LAYOUT, int CG>
 cudaError_t set_attr_one() {
-  if constexpr (!tc_supported<BN, EPI, LAYOUT>()) return cudaSuccess;
-  else return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcLayout<BN, EPI>::SMEM_BYTES);
+  if constexpr (!tc_supported<BN, EPI, LAYOUT, CG>()) return cudaSuccess;
+  else return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, LAYOUT, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcLayout<BN, EPI, CG>::SMEM_BYTES);
 }
 
-template <int BN, int LAYOUT>
+template <int BN, int LAYOUT, int CG>
 cudaError_t launch_bn(int epi, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
                       const CUtensorMap& tD, const GemmArgs& a, int num_sms, cudaStream_t s) {
   switch (epi) {
-    case EPI_BIAS: return launch_one<BN, EPI_BIAS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_GELU: return launch_one<BN, EPI_GELU, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_RESID: return launch_one<BN, EPI_RESID, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_BIAS: return launch_one<BN, EPI_BIAS, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_GELU: return launch_one<BN, EPI_GELU, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_RESID: return launch_one<BN, EPI_RESID, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
     case EPI_LMHEAD:
-      return a.out != nullptr ? launch_one<BN, EPI_LMHEAD_LOGITS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s)
-                              : launch_one<BN, EPI_LMHEAD, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_F32: return launch_one<BN, EPI_F32, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_DGELU: return launch_one<BN, EPI_DGELU, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_DLOGITS: return launch_one<BN, EPI_DLOGITS, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
-    case EPI_GELU_SAVE: return launch_one<BN, EPI_GELU_SAVE, LAYOUT>(tA, tB, tC, tD, a, num_sms, s);
+      return a.out != nullptr ? launch_one<BN, EPI_LMHEAD_LOGITS, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s)
+                              : launch_one<BN, EPI_LMHEAD, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_F32: return launch_one<BN, EPI_F32, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_DGELU: return launch_one<BN, EPI_DGELU, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_DLOGITS: return launch_one<BN, EPI_DLOGITS, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
+    case EPI_GELU_SAVE: return launch_one<BN, EPI_GELU_SAVE, LAYOUT, CG>(tA, tB, tC, tD, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
 
 template <int BN>
-cudaError_t launch_layout(int layout, int epi, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
-                          const CUtensorMap& tD, const GemmArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_layout(int layout, int pair, int epi, const CUtensorMap& tA, const CUtensorMap& tB,
+                          const CUtensorMap& tC, const CUtensorMap& tD, const GemmArgs& a, int num_sms,
+                          cudaStream_t s) {
+  if (pair) return layout == LAYOUT_KK ? launch_bn<BN, LAYOUT_KK, 2>(epi, tA, tB, tC, tD, a, num_sms, s)
+                                       : cudaErrorInvalidValue;
   switch (layout) {
-    case LAYOUT_KK: return launch_bn<BN, LAYOUT_KK>(epi, tA, tB, tC, tD, a, num_sms, s);
-    case LAYOUT_B_MN: return launch_bn<BN, LAYOUT_B_MN>(epi, tA, tB, tC, tD, a, num_sms, s);
-    case LAYOUT_MN_MN: return launch_bn<BN, LAYOUT_MN_MN>(epi, tA, tB, tC, tD, a, num_sms, s);
+    case LAYOUT_KK: return launch_bn<BN, LAYOUT_KK, 1>(epi, tA, tB, tC, tD, a, num_sms, s);
+    case LAYOUT_B_MN: return launch_bn<BN, LAYOUT_B_MN, 1>(epi, tA, tB, tC, tD, a, num_sms, s);
+    case LAYOUT_MN_MN: return launch_bn<BN, LAYOUT_MN_MN, 1>(epi, tA, tB, tC, tD, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -729,71 +847,93 @@ bool make_tmap_3d_f32(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d
 
 int gemm_tc_n_tiles(int N, int bn) { return (bn / 64) * ((N + bn - 1) / bn); }   // TcLayout::GROUPS per tile
 
-int gemm_tc_pick_bn(int M, int N, int num_sms, int epi) {
-  // The fp32 epilogues run with tiles of at most 192 columns.
-  const int max_bn = (epi == EPI_RESID || epi == EPI_F32) ? 192 : 256;
+bool gemm_tc_pair_ok(int epi, int layout, int bn) {
+  return layout == LAYOUT_KK && bn >= 128 && epi != EPI_F32 && epi != EPI_DGELU;
+}
+
+GemmPick gemm_tc_pick(int M, int N, int num_sms, int epi, int layout) {
+  // CTA pairs (K-major operands, at least two 128-row blocks, the forward
+  // and logits-gradient epilogues) only on request, G2_GEMM_PAIR=1: on the
+  // B200 they measured no faster on the GPT-2 shapes (the single-CTA main
+  // loop is not bound by shared-memory bandwidth; the block's GEMMs are
+  // bound by pipeline fill, the exposed last epilogue and whole waves of
+  // tiles, and the pair's two epilogues gate each other's accumulator).
+  bool pair = false;
+  if (const char* e = getenv("G2_GEMM_PAIR"))
+    pair = atoi(e) != 0 && layout == LAYOUT_KK && M > TC_BM && epi != EPI_F32 && epi != EPI_DGELU && num_sms >= 2;
+  // The fp32 epilogues run with tiles of at most 192 columns on one CTA.
+  const int max_bn = (!pair && (epi == EPI_RESID || epi == EPI_F32)) ? 192 : 256;
+  const int min_bn = pair ? 128 : 64;
   // G2_GEMM_BN=64|128|192|256 pins the tile width (tests use it to cover
   // every instantiation); otherwise the width is chosen by the cost model below.
   if (const char* e = getenv("G2_GEMM_BN")) {
     const int v = atoi(e);
-    if (v == 64 || v == 128 || v == 192 || v == 256) return v < max_bn ? v : max_bn;
+    if (v == 64 || v == 128 || v == 192 || v == 256) return GemmPick{std::max(std::min(v, max_bn), min_bn), pair};
   }
   // Estimated cost = waves x per-tile cost. Narrower tiles re-read A from
   // shared memory more often per FLOP (the 128-row MMA at N=128 runs at
   // about 60% of the N=256 rate), so their per-column cost is higher; N=192
   // still keeps the MMA's shared-memory reads under the per-SM bandwidth.
-  // A narrower width must win by more than 2% to be taken.
+  // A narrower width must win by more than 2% to be taken. A pair's tile is
+  // 256 rows and a wave is one tile per pair of SMs.
   const int cand[4] = {256, 192, 128, 64};
   const double unit[4] = {256.0, 192.0, 200.0, 150.0};
-  const int mt = (M + TC_BM - 1) / TC_BM;
+  const int bm = pair ? 2 * TC_BM : TC_BM;
+  const int slots = pair ? num_sms / 2 : num_sms;
+  const int mt = (M + bm - 1) / bm;
   int best = max_bn;
   double best_cost = 1e30;
   for (int i = 0; i < 4; ++i) {
-    if (cand[i] > max_bn) continue;
+    if (cand[i] > max_bn || cand[i] < min_bn) continue;
     const long tiles = (long)mt * ((N + cand[i] - 1) / cand[i]);
-    const long waves = (tiles + num_sms - 1) / num_sms;
+    const long waves = (tiles + slots - 1) / slots;
     const double cost = waves * unit[i];
     if (cost < best_cost * 0.98) {
       best_cost = cost;
       best = cand[i];
     }
   }
-  return best;
+  return GemmPick{best, pair};
 }
 
+int gemm_tc_pick_bn(int M, int N, int num_sms, int epi) { return gemm_tc_pick(M, N, num_sms, epi).bn; }
+
 cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tC,
-                           const GemmArgs& a, int num_sms, cudaStream_t s, int layout, const CUtensorMap* tD) {
+                           const GemmArgs& a, int num_sms, cudaStream_t s, int layout, const CUtensorMap* tD,
+                           int pair) {
   if (epi == EPI_GELU_SAVE && tD == nullptr) return cudaErrorInvalidValue;
+  if (pair && !gemm_tc_pair_ok(epi, layout, bn)) return cudaErrorInvalidValue;
   const CUtensorMap& d = tD ? *tD : tC;
   switch (bn) {
-    case 256: return launch_layout<256>(layout, epi, tA, tB, tC, d, a, num_sms, s);
-    case 192: return launch_layout<192>(layout, epi, tA, tB, tC, d, a, num_sms, s);
-    case 128: return launch_layout<128>(layout, epi, tA, tB, tC, d, a, num_sms, s);
-    case 64: return launch_layout<64>(layout, epi, tA, tB, tC, d, a, num_sms, s);
+    case 256: return launch_layout<256>(layout, pair, epi, tA, tB, tC, d, a, num_sms, s);
+    case 192: return launch_layout<192>(layout, pair, epi, tA, tB, tC, d, a, num_sms, s);
+    case 128: return launch_layout<128>(layout, pair, epi, tA, tB, tC, d, a, num_sms, s);
+    case 64: return launch_layout<64>(layout, pair, epi, tA, tB, tC, d, a, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
 
 namespace {
-template <int BN, int LAYOUT>
+template <int BN, int LAYOUT, int CG>
 cudaError_t set_attr_layout() {
   cudaError_t e = cudaSuccess;
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_BIAS, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD_LOGITS, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_F32, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_DGELU, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_DLOGITS, LAYOUT>();
-  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU_SAVE, LAYOUT>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_BIAS, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_RESID, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_LMHEAD_LOGITS, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_F32, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_DGELU, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_DLOGITS, LAYOUT, CG>();
+  if (e == cudaSuccess) e = set_attr_one<BN, EPI_GELU_SAVE, LAYOUT, CG>();
   return e;
 }
 template <int BN>
 cudaError_t set_attr_bn() {
-  cudaError_t e = set_attr_layout<BN, LAYOUT_KK>();
-  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_B_MN>();
-  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_MN_MN>();
+  cudaError_t e = set_attr_layout<BN, LAYOUT_KK, 1>();
+  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_B_MN, 1>();
+  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_MN_MN, 1>();
+  if (e == cudaSuccess) e = set_attr_layout<BN, LAYOUT_KK, 2>();
   return e;
 }
 }  // namespace

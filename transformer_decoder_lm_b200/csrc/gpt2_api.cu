@@ -122,8 +122,9 @@ int run_linear(gpt2_model* m, int epi, const void* A, const CUtensorMap* tmA, co
   if (m->bf16 && M <= GEMV_MAX_M) {   // a few rows (decoding): one warp per output column
     e = gemv_bf16_launch(epi, A, W, a, s);
   } else if (m->bf16) {
-    const int bn = gemm_tc_pick_bn(M, N, m->num_sms, epi);
-    e = gemm_tc_launch(epi, bn, *tmA, wmaps[bn_index(bn)], *tmC, a, m->num_sms, s);
+    const GemmPick p = gemm_tc_pick(M, N, m->num_sms, epi);
+    e = gemm_tc_launch(epi, p.bn, *tmA, wmaps[box_index(gemm_tc_b_box_rows(p))], *tmC, a, m->num_sms, s, LAYOUT_KK,
+                       nullptr, p.pair);
   } else {
     e = gemm_simt_launch(epi, static_cast<const float*>(A), static_cast<const float*>(W), a, s);
   }
@@ -218,9 +219,10 @@ int run_forward(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B
     int n_tiles;
     if (m->ev_lm_begin) G2_CK(cudaEventRecord(m->ev_lm_begin, s));
     if (m->bf16) {
-      const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
-      n_tiles = gemm_tc_n_tiles(V, bn);
-      G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, tm_h, m->wte_map[bn_index(bn)], tm_h, a, m->num_sms, s));
+      const GemmPick p = lmhead_pick(M, V, m->num_sms);
+      n_tiles = gemm_tc_n_tiles(V, p.bn);
+      G2_CK(gemm_tc_launch(EPI_LMHEAD, p.bn, tm_h, m->wte_map[box_index(gemm_tc_b_box_rows(p))], tm_h, a,
+                           m->num_sms, s, LAYOUT_KK, nullptr, p.pair));
     } else {
       n_tiles = (V + SIMT_BN - 1) / SIMT_BN;
       G2_CK(gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(m->h), static_cast<const float*>(m->wte), a, s));
@@ -318,8 +320,9 @@ int run_decode(gpt2_model* m, void* kv_cache, const int32_t* ids, int B, int pos
   a.tgt_logit = m->tgt;
   a.status = m->status;
   if (m->bf16) {
-    const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
-    G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, tm_h, m->wte_map[bn_index(bn)], tm_h, a, m->num_sms, s));
+    const GemmPick p = lmhead_pick(M, V, m->num_sms);
+    G2_CK(gemm_tc_launch(EPI_LMHEAD, p.bn, tm_h, m->wte_map[box_index(gemm_tc_b_box_rows(p))], tm_h, a, m->num_sms,
+                         s, LAYOUT_KK, nullptr, p.pair));
   } else {
     G2_CK(gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(m->h), static_cast<const float*>(m->wte), a, s));
   }
@@ -358,11 +361,12 @@ cudaError_t g2::lmhead_ce_launch(bool bf16, const void* hf, const void* wte, con
   int n_groups;
   cudaError_t e;
   if (bf16) {
-    const int bn = std::max(gemm_tc_pick_bn(M, V, sms, EPI_LMHEAD), LMHEAD_MIN_BN);
-    n_groups = gemm_tc_n_tiles(V, bn);
+    const GemmPick p = lmhead_pick(M, V, sms);
+    n_groups = gemm_tc_n_tiles(V, p.bn);
     CUtensorMap ta, tb;
-    if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return cudaErrorInvalidValue;
-    e = gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, ta, a, sms, s);
+    if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, gemm_tc_b_box_rows(p)))
+      return cudaErrorInvalidValue;
+    e = gemm_tc_launch(EPI_LMHEAD, p.bn, ta, tb, ta, a, sms, s, LAYOUT_KK, nullptr, p.pair);
   } else {
     n_groups = (V + SIMT_BN - 1) / SIMT_BN;
     e = gemm_simt_launch(EPI_LMHEAD, static_cast<const float*>(hf), static_cast<const float*>(wte), a, s);
@@ -454,8 +458,8 @@ int gpt2_create(const gpt2_config_t* cfg, const gpt2_weights_t* w, void* workspa
     const int C = cfg->n_embd;
     m->maps.resize(L);
     bool ok = true;
-    for (int i = 0; i < NUM_BN && ok; ++i) {
-      const uint32_t bn = BN_CHOICES[i];
+    for (int i = 0; i < NUM_BOX && ok; ++i) {
+      const uint32_t bn = BOX_ROWS[i];
       ok = ok && make_tmap_bf16(&m->wte_map[i], m->wte, cfg->vocab, C, C, bn);
       for (int l = 0; l < L && ok; ++l) {
         ok = ok && make_tmap_bf16(&m->maps[l].attn[i], m->layers[l].attn_w, 3 * C, C, C, bn);
@@ -608,13 +612,16 @@ int gpt2_op_linear(int dtype, int epilogue, const void* A, const void* W, const 
   int sms = 0;
   int rc = device_setup(nullptr, &sms);
   if (rc != GPT2_OK) return rc;
-  const int bn = gemm_tc_pick_bn(M, N, sms, epilogue);
+  const GemmPick p = gemm_tc_pick(M, N, sms, epilogue);
   CUtensorMap ta, tb, tc;
-  if (!make_tmap_bf16(&ta, A, M, K, K, 128) || !make_tmap_bf16(&tb, W, N, K, K, bn)) return GPT2_ERR_CUDA;
+  if (!make_tmap_bf16(&ta, A, M, K, K, 128) || !make_tmap_bf16(&tb, W, N, K, K, gemm_tc_b_box_rows(p)))
+    return GPT2_ERR_CUDA;
   const bool ok_c = epilogue == GPT2_EPI_BIAS_RESID ? make_tmap_out_f32(&tc, out, M, N, N)
                                                      : make_tmap_out_bf16(&tc, out, M, N, N);
   if (!ok_c) return GPT2_ERR_CUDA;
-  return gemm_tc_launch(epilogue, bn, ta, tb, tc, a, sms, s) == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+  return gemm_tc_launch(epilogue, p.bn, ta, tb, tc, a, sms, s, LAYOUT_KK, nullptr, p.pair) == cudaSuccess
+             ? GPT2_OK
+             : GPT2_ERR_CUDA;
 }
 
 int gpt2_op_embed_layernorm(const int32_t* ids, const void* wte, const void* wpe, int M, int T, int C, int V,

@@ -86,7 +86,7 @@ bool make_tmap_3d_f32(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d
                       uint64_t s2, uint32_t box0, uint32_t box1);
 // Column groups of lm_head partials for N columns (two per tile of width bn).
 int gemm_tc_n_tiles(int N, int bn);
-// The lm_head runs with tiles of at least this width.
+// The lm_head runs with tiles of at least this width (lmhead_pick).
 constexpr int LMHEAD_MIN_BN = 128;
 // lm_head partials per row: one per 64-column group of a tcgen05 tile (tiles
 // of BN columns cover V padded up to a multiple of BN) or per 64-column SIMT
@@ -111,10 +111,27 @@ cudaError_t lmhead_ce_launch(bool bf16, const void* hf, const void* wte, const i
 // 64 x 64 (make_tmap_bf16 with box_rows 64). tmC: the output map
 // (make_tmap_out_*; unused by EPI_LMHEAD); tmD: EPI_GELU_SAVE's
 // pre-activation output (bf16, like tmC).
-int gemm_tc_pick_bn(int M, int N, int num_sms, int epi);
+// pair = 1: CTA pairs (clusters of two) compute 256 x BN tiles with one
+// M = 256 tcgen05.mma; each CTA loads half of B, so tmB's box is BN / 2 rows
+// (K-major operands, BN >= 128, not EPI_F32 / EPI_DGELU: gemm_tc_pair_ok).
+struct GemmPick {
+  int bn;     // tile width
+  int pair;   // 1: CTA pairs
+};
+GemmPick gemm_tc_pick(int M, int N, int num_sms, int epi, int layout = LAYOUT_KK);
+int gemm_tc_pick_bn(int M, int N, int num_sms, int epi);   // gemm_tc_pick(...).bn
+bool gemm_tc_pair_ok(int epi, int layout, int bn);
+// Rows of tmB's box for a pick: BN, or BN / 2 for a pair.
+inline int gemm_tc_b_box_rows(const GemmPick& p) { return p.pair ? p.bn / 2 : p.bn; }
+// The lm_head's pick: gemm_tc_pick with tiles of at least LMHEAD_MIN_BN.
+inline GemmPick lmhead_pick(int M, int V, int num_sms) {
+  GemmPick p = gemm_tc_pick(M, V, num_sms, EPI_LMHEAD);
+  if (p.bn < LMHEAD_MIN_BN) p.bn = LMHEAD_MIN_BN;
+  return p;
+}
 cudaError_t gemm_tc_launch(int epi, int bn, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
                            const GemmArgs& a, int num_sms, cudaStream_t s, int layout = LAYOUT_KK,
-                           const CUtensorMap* tmD = nullptr);
+                           const CUtensorMap* tmD = nullptr, int pair = 0);
 cudaError_t gemm_tc_set_attributes();
 
 // ---- SIMT fp32 GEMM (fp32 mode) ------------------------------------------

@@ -13,9 +13,13 @@
 
 namespace g2 {
 
-constexpr int NUM_BN = 4;
-constexpr int BN_CHOICES[NUM_BN] = {256, 192, 128, 64};
-inline int bn_index(int bn) { return bn == 256 ? 0 : (bn == 192 ? 1 : (bn == 128 ? 2 : 3)); }
+// Weight tensor maps are kept for every box height a GEMM pick can ask for:
+// the tile widths (single CTA) and their halves (CTA pairs: 96 for 192).
+constexpr int NUM_BOX = 5;
+constexpr int BOX_ROWS[NUM_BOX] = {256, 192, 128, 96, 64};
+inline int box_index(int rows) {
+  return rows == 256 ? 0 : (rows == 192 ? 1 : (rows == 128 ? 2 : (rows == 96 ? 3 : 4)));
+}
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -25,8 +29,8 @@ struct LayerPtrs {
   const void *ln2_g, *ln2_b, *fc_w, *fc_b, *mlp_proj_w, *mlp_proj_b;
 };
 
-struct WeightMaps {  // one tensor map per candidate tile width
-  CUtensorMap attn[NUM_BN], proj[NUM_BN], fc[NUM_BN], mproj[NUM_BN];
+struct WeightMaps {  // one tensor map per box height
+  CUtensorMap attn[NUM_BOX], proj[NUM_BOX], fc[NUM_BOX], mproj[NUM_BOX];
 };
 
 // Byte offsets of the workspace slices (gpt2_create).
@@ -46,7 +50,7 @@ struct gpt2_model {
   const void *wte = nullptr, *wpe = nullptr, *lnf_g = nullptr, *lnf_b = nullptr;
   std::vector<g2::LayerPtrs> layers;
   std::vector<g2::WeightMaps> maps;
-  CUtensorMap wte_map[g2::NUM_BN];
+  CUtensorMap wte_map[g2::NUM_BOX];
   uint8_t* ws = nullptr;
   g2::Plan plan;
   float* x = nullptr;

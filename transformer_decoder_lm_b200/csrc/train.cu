@@ -104,11 +104,13 @@ struct Gemm {
   int run(int epi, const void* A, bool a_mn, long long lda, const void* B, bool b_mn, long long ldb, void* out,
           long long ldo, bool out_f32, int M, int N, int K, const GemmArgs& extra = GemmArgs{},
           const void* out_d = nullptr, int b_rows = -1) const {
-    const int bn = gemm_tc_pick_bn(M, N, sms, epi == EPI_DLOGITS ? EPI_LMHEAD : epi);
+    const int layout = (a_mn ? LAYOUT_A_MN : 0) | (b_mn ? LAYOUT_B_MN : 0);
+    const GemmPick p = gemm_tc_pick(M, N, sms, epi == EPI_DLOGITS ? EPI_LMHEAD : epi, layout);
+    const int bn = p.bn;
     CUtensorMap ta, tb, tc, td;
     const bool ok_a = a_mn ? make_tmap_bf16(&ta, A, K, M, lda, 64) : make_tmap_bf16(&ta, A, M, K, lda, 128);
     const bool ok_b = b_mn ? make_tmap_bf16(&tb, B, b_rows > 0 ? std::min(b_rows, K) : K, N, ldb, 64)
-                           : make_tmap_bf16(&tb, B, N, K, ldb, bn);
+                           : make_tmap_bf16(&tb, B, N, K, ldb, gemm_tc_b_box_rows(p));
     const bool ok_c = out_f32 ? make_tmap_out_f32(&tc, out, M, N, ldo) : make_tmap_out_bf16(&tc, out, M, N, ldo);
     const bool ok_d = out_d == nullptr || make_tmap_out_bf16(&td, out_d, M, N, ldo);
     if (!ok_a || !ok_b || !ok_c || !ok_d) return GPT2_ERR_CUDA;
@@ -126,8 +128,7 @@ struct Gemm {
       a.k_split = 2;
       if (cudaMemset2DAsync(out, (size_t)ldo * 4, 0, (size_t)N * 4, M, s) != cudaSuccess) return GPT2_ERR_CUDA;
     }
-    const int layout = (a_mn ? LAYOUT_A_MN : 0) | (b_mn ? LAYOUT_B_MN : 0);
-    return gemm_tc_launch(epi, bn, ta, tb, tc, a, sms, s, layout, out_d ? &td : nullptr) == cudaSuccess
+    return gemm_tc_launch(epi, bn, ta, tb, tc, a, sms, s, layout, out_d ? &td : nullptr, p.pair) == cudaSuccess
                ? GPT2_OK
                : GPT2_ERR_CUDA;
   }
@@ -219,15 +220,16 @@ int run_train(gpt2_model* m, const int32_t* ids, const int32_t* targets, int B, 
     a.targets = targets;
     a.part = m->part;
     a.tgt_logit = m->tgt;
-    const int bn = std::max(gemm_tc_pick_bn(M, V, m->num_sms, EPI_LMHEAD), LMHEAD_MIN_BN);
+    const GemmPick p = lmhead_pick(M, V, m->num_sms);
     CUtensorMap ta;
     if (!make_tmap_bf16(&ta, hf, M, C, C, 128)) return GPT2_ERR_CUDA;
     a.M = M;
     a.N = V;
     a.K = C;
     a.status = m->status;
-    G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, ta, m->wte_map[bn_index(bn)], ta, a, m->num_sms, s));
-    G2_CK(ce_finish_launch(m->part, gemm_tc_n_tiles(V, bn), m->tgt, targets, M, V, m->tok, loss_out, m->status, s,
+    G2_CK(gemm_tc_launch(EPI_LMHEAD, p.bn, ta, m->wte_map[box_index(gemm_tc_b_box_rows(p))], ta, a, m->num_sms, s,
+                         LAYOUT_KK, nullptr, p.pair));
+    G2_CK(ce_finish_launch(m->part, gemm_tc_n_tiles(V, p.bn), m->tgt, targets, M, V, m->tok, loss_out, m->status, s,
                            lse_ce, n_scored));
   }
 
@@ -461,11 +463,12 @@ int gpt2_op_lmhead_ce_backward(const void* hf, const void* wte, const int32_t* t
   a.part = part;
   a.tgt_logit = tgt;
   a.status = status;
-  const int bn = std::max(gemm_tc_pick_bn(M, V, sms, EPI_LMHEAD), LMHEAD_MIN_BN);
+  const GemmPick p = lmhead_pick(M, V, sms);
   CUtensorMap ta, tb;
-  if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, bn)) return GPT2_ERR_CUDA;
-  G2_CK(gemm_tc_launch(EPI_LMHEAD, bn, ta, tb, ta, a, sms, s));
-  G2_CK(ce_finish_launch(part, gemm_tc_n_tiles(V, bn), tgt, targets, M, V, tok, loss_out, status, s, lse, n_scored));
+  if (!make_tmap_bf16(&ta, hf, M, C, C, 128) || !make_tmap_bf16(&tb, wte, V, C, C, gemm_tc_b_box_rows(p)))
+    return GPT2_ERR_CUDA;
+  G2_CK(gemm_tc_launch(EPI_LMHEAD, p.bn, ta, tb, ta, a, sms, s, LAYOUT_KK, nullptr, p.pair));
+  G2_CK(ce_finish_launch(part, gemm_tc_n_tiles(V, p.bn), tgt, targets, M, V, tok, loss_out, status, s, lse, n_scored));
   const Gemm gm{sms, status, s};
   GemmArgs d{};
   d.targets = targets;
