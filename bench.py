@@ -6,7 +6,9 @@ One step = one full forward pass through the C ABI (gpt2_forward_loss):
 embedding, 12 Pre-LN blocks, ln_f, the tied lm_head writing fp32 logits
 [4, 1024, 50257], and the shifted cross-entropy. Inputs are resident in HBM
 when the timed region starts; `e2e` repeats the measurement with the ids and
-targets copied from pinned host memory and the loss read back every step.
+targets copied from pinned host memory and the loss read back every step
+(the copies on a second stream, overlapping the neighbouring steps;
+`serial_value`: the same with every copy between the steps).
 Under torchrun (N > 1) every rank runs its own batch of 4 sequences (weak
 scaling, data-parallel replicas); the only exchange is an all-reduce of the
 loss numerator and count. Rank 0 prints one JSON line.
@@ -251,10 +253,11 @@ def run_ours(args):
 
     from transformer_decoder_lm_b200 import dist as gdist
 
-    def step(i_ids, i_tg):
-        G.gpt2_forward_loss(model.handle, i_ids, i_tg, WL.batch, WL.seq, logits, loss, None, stream)
+    def step(i_ids, i_tg, o_loss=None):
+        o_loss = loss if o_loss is None else o_loss
+        G.gpt2_forward_loss(model.handle, i_ids, i_tg, WL.batch, WL.seq, logits, o_loss, None, stream)
         if world > 1:   # the one exchange of the data-parallel forward: the loss mean
-            loss.copy_(gdist.global_mean_loss(loss, int(n_valid)))
+            o_loss.copy_(gdist.global_mean_loss(o_loss, int(n_valid)))
 
     def barrier():
         if world > 1:
@@ -334,33 +337,74 @@ def run_ours(args):
     if rc != 0:
         raise RuntimeError(f"device status after the variants: {G.gpt2_error_string(rc)}")
 
-    # e2e: host buffers, copies inside the timed region
+    # e2e: host buffers, copies inside the timed region: every step copies
+    # its ids and targets from pinned host memory and reads its loss back.
+    # As a production loop does, the copies run on a second stream, double
+    # buffered: step i+1's inputs go up while step i computes, and step i's
+    # loss comes back while step i+1 runs; the timed region ends after the
+    # last loss has reached the host. The same loop with every copy on the
+    # compute stream, between the steps, is reported as e2e_serial.
     h_ids = torch.from_numpy(ids_np).pin_memory()
     h_tg = torch.from_numpy(tg_np).pin_memory()
-    h_loss = torch.empty(1, dtype=torch.float32).pin_memory()
-    d_ids = torch.empty_like(ids)
-    d_tg = torch.empty_like(tg)
+    h_loss = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(2)]
+    d_ids = [torch.empty_like(ids) for _ in range(2)]
+    d_tg = [torch.empty_like(tg) for _ in range(2)]
+    d_loss = [torch.empty(1, dtype=torch.float32, device="cuda") for _ in range(2)]
+    cs = torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_read = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        d_ids.copy_(h_ids, non_blocking=True)
-        d_tg.copy_(h_tg, non_blocking=True)
-        step(d_ids, d_tg)
-        h_loss.copy_(loss, non_blocking=True)
+    def e2e_pipelined(n):
+        with torch.cuda.stream(cs):
+            d_ids[0].copy_(h_ids, non_blocking=True)
+            d_tg[0].copy_(h_tg, non_blocking=True)
+            ev_in[0].record(cs)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:   # the next step's inputs, once step i-1 no longer reads that buffer
+                with torch.cuda.stream(cs):
+                    if i >= 1:
+                        cs.wait_event(ev_done[b ^ 1])
+                    d_ids[b ^ 1].copy_(h_ids, non_blocking=True)
+                    d_tg[b ^ 1].copy_(h_tg, non_blocking=True)
+                    ev_in[b ^ 1].record(cs)
+            stream.wait_event(ev_in[b])
+            if i >= 2:   # step i-2's loss has been read out of this buffer
+                stream.wait_event(ev_read[b])
+            step(d_ids[b], d_tg[b], d_loss[b])
+            ev_done[b].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_done[b])
+                h_loss[b].copy_(d_loss[b], non_blocking=True)
+                ev_read[b].record(cs)
+        stream.wait_stream(cs)
 
-    for _ in range(3):
-        e2e_step()
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    barrier()
-    ems = e0.elapsed_time(e1)
-    if world > 1:
-        ems = gdist.max_over_ranks(ems, "cuda")
-    e2e_value = tokens_all / (ems / args.steps / 1000.0)
+    def e2e_serial(n):
+        for _ in range(n):
+            d_ids[0].copy_(h_ids, non_blocking=True)
+            d_tg[0].copy_(h_tg, non_blocking=True)
+            step(d_ids[0], d_tg[0], d_loss[0])
+            h_loss[0].copy_(d_loss[0], non_blocking=True)
+
+    def timed_e2e(run):
+        run(3)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(args.steps)
+        e1.record(stream)
+        barrier()
+        t = e0.elapsed_time(e1)
+        if world > 1:
+            t = gdist.max_over_ranks(t, "cuda")
+        return tokens_all / (t / args.steps / 1000.0)
+
+    e2e_value = timed_e2e(e2e_pipelined)
+    e2e_serial_value = timed_e2e(e2e_serial)
+    if not math.isfinite(float(h_loss[0].item())) or abs(float(h_loss[0].item()) - float(loss.item())) > 1e-5:
+        raise RuntimeError("the loss read back in the end-to-end loop differs from the device-timed one")
 
     hbm, tf_burst, tf_sust, peak_kind = peaks()
     lm_tflops = lmhead_flops(WL, M) / (lm_ms / 1000.0) / 1e12
@@ -383,7 +427,8 @@ def run_ours(args):
                      "launches_timed": lm_steps,
                      "peak_kind": f"{peak_kind} burst (the timed region lasts tens of milliseconds)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h_ids.numel() * 4 + h_tg.numel() * 4),
-                "d2h_bytes_per_step": 4},
+                "d2h_bytes_per_step": 4, "copies": "second stream, double buffered",
+                "serial_value": e2e_serial_value},
         "gpu_launches": int(launches),
         "variants": variants,
         "clocks": clk,
