@@ -72,9 +72,12 @@ struct TcLayout {
   static constexpr int B_ROWS = BN / CG;
   static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  // a single CTA keeps a 4-deep ring; a pair's smaller stages buy up to 6
+  // a single CTA keeps a 4-deep ring (3-deep for fp32 output at BN = 256,
+  // whose 4 KB staging per warp takes the fourth stage's room); a pair's
+  // smaller stages buy up to 6
   static constexpr int STAGES_FIT = (TC_SMEM_MAX - 1024 - 256 - EPI_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = CG == 1 ? TC_STAGES : (STAGES_FIT < 6 ? STAGES_FIT : 6);
+  static constexpr int STAGES =
+      CG == 1 ? (F32_OUT && BN == 256 ? 3 : TC_STAGES) : (STAGES_FIT < 6 ? STAGES_FIT : 6);
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, tmem_full[2], tmem_empty[2], drain
@@ -691,16 +694,19 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
 }
 
 
-// The fp32 epilogues' 4 KB staging per warp does not fit next to a single
-// CTA's ring at BN = 256 (gemm_tc_pick never picks it there). The backward
-// layouts are instantiated only with the epilogues the backward pass uses;
-// CTA pairs with K-major operands, 128 to 256 columns and the forward (and
-// logits-gradient) epilogues.
+// The fp32 epilogues' 4 KB staging per warp leaves room for a 3-deep ring at
+// BN = 256 on a single CTA: instantiated for the weight gradient (both
+// operands MN-major, the widest tiles whose K halves fill the SMs; the
+// residual epilogue keeps BN <= 192). The backward layouts are instantiated
+// only with the epilogues the backward pass uses; CTA pairs with K-major
+// operands, 128 to 256 columns and the forward (and logits-gradient)
+// epilogues.
 template <int BN, int EPI, int LAYOUT, int CG>
 constexpr bool tc_supported() {
   if (CG == 2)
     return LAYOUT == LAYOUT_KK && BN >= 128 && EPI != EPI_F32 && EPI != EPI_DGELU;
-  if ((EPI == EPI_RESID || EPI == EPI_F32) && BN == 256) return false;
+  if (EPI == EPI_RESID && BN == 256) return false;
+  if (EPI == EPI_F32 && BN == 256 && LAYOUT != LAYOUT_MN_MN) return false;
   if (LAYOUT == LAYOUT_B_MN) return EPI == EPI_BIAS || EPI == EPI_F32 || EPI == EPI_DGELU;
   if (LAYOUT == LAYOUT_MN_MN) return EPI == EPI_F32;
   if (LAYOUT == LAYOUT_A_MN) return false;

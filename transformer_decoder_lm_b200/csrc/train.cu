@@ -105,7 +105,31 @@ struct Gemm {
           long long ldo, bool out_f32, int M, int N, int K, const GemmArgs& extra = GemmArgs{},
           const void* out_d = nullptr, int b_rows = -1) const {
     const int layout = (a_mn ? LAYOUT_A_MN : 0) | (b_mn ? LAYOUT_B_MN : 0);
-    const GemmPick p = gemm_tc_pick(M, N, sms, epi == EPI_DLOGITS ? EPI_LMHEAD : epi, layout);
+    GemmPick p = gemm_tc_pick(M, N, sms, epi == EPI_DLOGITS ? EPI_LMHEAD : epi, layout);
+    // A weight gradient over many tokens (fp32 out, both operands MN-major)
+    // may run as two K halves added into a zeroed output when twice its tiles
+    // fit on the SMs: among the widths that allow that, the one with the
+    // least estimated time (waves x K per item x the width's cost per
+    // k-block, as in gemm_tc_pick), if it beats the pick without halves.
+    const bool wgrad = epi == EPI_F32 && a_mn && b_mn && out_f32 && K >= 1024;
+    bool halves = false;
+    if (wgrad) {
+      const int mt = (M + 127) / 128;
+      auto cost = [&](int w, int split) {
+        const long t = (long)mt * ((N + w - 1) / w) * split;
+        const double unit = w == 256 ? 256.0 : (w == 192 ? 192.0 : (w == 128 ? 200.0 : 150.0));
+        return (double)((t + sms - 1) / sms) * ((double)K / split) * unit;
+      };
+      double best = cost(p.bn, 1);
+      for (int w : {256, 192, 128, 64}) {
+        if (2L * mt * ((N + w - 1) / w) > sms) continue;
+        if (cost(w, 2) < best) {
+          best = cost(w, 2);
+          p.bn = w;
+          halves = true;
+        }
+      }
+    }
     const int bn = p.bn;
     CUtensorMap ta, tb, tc, td;
     const bool ok_a = a_mn ? make_tmap_bf16(&ta, A, K, M, lda, 64) : make_tmap_bf16(&ta, A, M, K, lda, 128);
@@ -121,10 +145,9 @@ struct Gemm {
     a.out = out;
     a.ldo = ldo;
     a.status = status;
-    // A weight gradient with too few tiles for the SMs and a long K (the
-    // tokens): the K range in two halves, both added into the zeroed output.
-    const long tiles = (long)((M + 127) / 128) * ((N + bn - 1) / bn);
-    if (epi == EPI_F32 && a_mn && b_mn && out_f32 && 2 * tiles <= sms && K >= 1024) {
+    // the K range in two halves, both added into the zeroed output (0 + a + b:
+    // the same bits in either order)
+    if (halves) {
       a.k_split = 2;
       if (cudaMemset2DAsync(out, (size_t)ldo * 4, 0, (size_t)N * 4, M, s) != cudaSuccess) return GPT2_ERR_CUDA;
     }
