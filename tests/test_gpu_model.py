@@ -61,6 +61,33 @@ def test_small_bf16_case_spans_tiles_and_tails(G):
     assert tie >= _cmp.BF16_TOP1
 
 
+@pytest.mark.parametrize("B,T", [(1, 1), (3, 1), (2, 5), (1, 17), (1, 256), (8, 2)])
+def test_degenerate_and_edge_shapes(G, B, T):
+    """A single position (no scored target: logits only), a batch of a few
+    rows (M <= 16: the few-row GEMV path with separate LayerNorms), one row
+    past it (M = 17: the tensor-core path with one ragged 128-row tile), a
+    sequence of the full context n_ctx, and many sequences of two positions
+    (one scored position each) against the oracle."""
+    wl = SMALL.scaled(batch=B, seq=T)
+    W = synthetic.make_weights(wl)
+    ids = synthetic.make_ids(wl)
+    model = G.GPT2Model.from_workload(wl, W)
+    d_ids = torch.from_numpy(ids).cuda()
+    ref = O.forward(W, ids, wl.n_head)
+    z = model.forward(d_ids).cpu().numpy()
+    assert model.status() == 0
+    assert z.shape == (B, T, wl.vocab)
+    assert _cmp.rel_l2(z, ref) <= _cmp.BF16_REL_L2
+    assert _cmp.max_abs(z, ref) <= _cmp.BF16_MAX_ABS
+    if T >= 2:
+        ref_loss, _ = O.shifted_cross_entropy(ref, ids)
+        d_tg = torch.from_numpy(synthetic.next_token_targets(ids)).cuda()
+        z2, loss = model.forward_loss(d_ids, d_tg)
+        assert model.status() == 0
+        assert torch.equal(z2.cpu(), torch.from_numpy(z))
+        assert abs(loss.item() - ref_loss) <= _cmp.BF16_LOSS_ABS
+
+
 def test_small_case_all_fp32_debug_mode(G):
     W, ids, model, z, loss, tok = run_case(G, SMALL, dtype="fp32")
     ref = O.forward(W, ids, SMALL.n_head)
