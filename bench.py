@@ -46,11 +46,13 @@ def n_params(wl) -> int:
 
 
 def model_flops(wl, tokens_per_seq=None, seqs=None) -> float:
-    """2 * params * tokens + causal attention 2 * C * T * (T + 1) per layer and
-    sequence (QK^T and PV over the lower triangle with its diagonal)."""
+    """2 * params * tokens over the parameters that multiply (every parameter
+    but the position table, which is gathered: the blocks, ln_f and the tied
+    wte as the lm_head), plus causal attention 2 * C * T * (T + 1) per layer
+    and sequence (QK^T and PV over the lower triangle with its diagonal)."""
     T = tokens_per_seq or wl.seq
     Bn = seqs or wl.batch
-    return 2.0 * n_params(wl) * Bn * T + wl.n_layer * Bn * 2.0 * wl.n_embd * T * (T + 1)
+    return 2.0 * (n_params(wl) - wl.n_ctx * wl.n_embd) * Bn * T + wl.n_layer * Bn * 2.0 * wl.n_embd * T * (T + 1)
 
 
 def lmhead_flops(wl, M) -> float:
